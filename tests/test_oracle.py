@@ -1,0 +1,276 @@
+"""Pins for the fp64 oracle, against facts other than the oracle itself.
+
+Each check follows from the linear-attention definition on page
+"MiniMax-M1で理解する：大規模言語モデルのコンテキスト長限界を突破する革新的アーキテクチャ"
+(zenn.dev), section "線形アテンションの数学的基礎" (S_t = S_{t-1} + k_t v_t^T,
+o_t = q_t S_t), from its factorised form phi(Q)(phi(K)^T V), or from plain
+linear algebra: a hand-worked fixture, brute force over token pairs, closed
+forms through numpy, integer exactness and invariants.  The mutant tests at
+the end plant plausible mistakes in copies of the oracle's formulas and show
+that these pins reject them.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _read_golden(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            rows[key] = np.array([float(x) for x in vals])
+    return rows
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+# ---------------------------------------------------------------- fixtures
+def test_hand_worked_example(oracle_mod):
+    g = _read_golden("hand_worked_n3_d2.txt")
+    q = g["q"].reshape(1, 3, 2)
+    k = g["k"].reshape(1, 3, 2)
+    v = g["v"].reshape(1, 3, 2)
+    for fn in (oracle_mod.recurrent, oracle_mod.quadratic):
+        o, s = fn(q, k, v)
+        np.testing.assert_array_equal(o.reshape(-1), g["A.o"])
+        np.testing.assert_array_equal(s.reshape(-1), g["A.S"])
+        s0 = g["B.S0"].reshape(1, 2, 2)
+        o, s = fn(q, k, v, s0)
+        np.testing.assert_array_equal(o.reshape(-1), g["B.o"])
+        np.testing.assert_array_equal(s.reshape(-1), g["B.S"])
+
+
+def _brute(q, k, v, s0):
+    """o_t = sum_{s<=t} (q_t . k_s) v_s + q_t S0 and S_N = S0 + sum_s k_s^T v_s,
+    written as explicit pure-Python loops over token pairs."""
+    N, dk = q.shape
+    dv = v.shape[1]
+    o = [[0.0] * dv for _ in range(N)]
+    for t in range(N):
+        for s in range(t + 1):
+            a = sum(float(q[t, i]) * float(k[s, i]) for i in range(dk))
+            for j in range(dv):
+                o[t][j] += a * float(v[s, j])
+        for j in range(dv):
+            o[t][j] += sum(float(q[t, i]) * float(s0[i, j]) for i in range(dk))
+    S = [[float(s0[i, j]) + sum(float(k[s, i]) * float(v[s, j]) for s in range(N))
+          for j in range(dv)] for i in range(dk)]
+    return np.array(o), np.array(S)
+
+
+@pytest.mark.parametrize("N,dk,dv", [(1, 3, 2), (2, 4, 4), (5, 3, 6), (8, 8, 8), (7, 2, 5)])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_brute_force_small(oracle_mod, N, dk, dv, with_s0):
+    q = _rand((N, dk), 1)
+    k = _rand((N, dk), 2)
+    v = _rand((N, dv), 3)
+    s0 = _rand((dk, dv), 4) if with_s0 else np.zeros((dk, dv))
+    ob, sb = _brute(q, k, v, s0)
+    for fn in (oracle_mod.recurrent, oracle_mod.quadratic):
+        o, s = fn(q[None], k[None], v[None], s0[None] if with_s0 else None)
+        assert _rel(o[0], ob) < 1e-13
+        assert _rel(s[0], sb) < 1e-13
+
+
+@pytest.mark.parametrize("N,d", [(256, 64), (300, 128), (129, 128), (1024, 64)])
+def test_recurrent_equals_quadratic(oracle_mod, N, d):
+    q, k, v = synth.qkv((2, 2, N, d), d, "fp32", seed=N + d)
+    s0 = _rand((2, 2, d, d), 7)
+    o1, s1 = oracle_mod.recurrent(q, k, v, s0)
+    o2, s2 = oracle_mod.quadratic(q, k, v, s0)
+    assert _rel(o1, o2) < 1e-12
+    assert _rel(s1, s2) < 1e-12
+
+
+def test_first_output_invariant(oracle_mod):
+    """o_1 = (q_1 . k_1) v_1 with a zero initial state; o_1 = q_1 S0 + (q_1 . k_1) v_1 otherwise."""
+    q, k, v = synth.qkv((3, 5, 64), 64, "fp32", seed=11)
+    o, _ = oracle_mod.recurrent(q, k, v)
+    qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+    want = np.einsum("ui,ui->u", qn[:, 0], kn[:, 0])[:, None] * vn[:, 0]
+    assert _rel(o[:, 0], want) < 1e-14
+    s0 = _rand((3, 64, 64), 5)
+    o, _ = oracle_mod.recurrent(q, k, v, s0)
+    want2 = want + np.einsum("ui,uij->uj", qn[:, 0], s0)
+    assert _rel(o[:, 0], want2) < 1e-14
+
+
+def test_integer_inputs_exact(oracle_mod):
+    """Inputs in {-1,0,1}: every partial sum is a small integer, so both forms are exact."""
+    shape = (2, 3, 200, 16)
+    q = synth.integer_valued(shape, seed=1)
+    k = synth.integer_valued(shape, seed=2)
+    v = synth.integer_valued(shape, seed=3)
+    s0 = synth.integer_valued((2, 3, 16, 16), seed=4, lo=-3, hi=3)
+    o1, s1 = oracle_mod.recurrent(q, k, v, s0)
+    o2, s2 = oracle_mod.quadratic(q, k, v, s0)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+    assert np.all(o1 == np.round(o1))
+    # exact brute force on one unit
+    ob, sb = _brute(q[1, 2].numpy(), k[1, 2].numpy(), v[1, 2].numpy(), s0[1, 2].numpy())
+    np.testing.assert_array_equal(o1[1, 2], ob)
+    np.testing.assert_array_equal(s1[1, 2], sb)
+
+
+def test_final_state_is_library_gemm(oracle_mod):
+    """S_N = S0 + K^T V, checked against numpy's matmul."""
+    q, k, v = synth.qkv((4, 333, 32), 48, "fp32", seed=3)
+    s0 = _rand((4, 32, 48), 9)
+    _, s = oracle_mod.recurrent(q, k, v, s0)
+    kn, vn = k.double().numpy(), v.double().numpy()
+    want = s0 + np.matmul(kn.transpose(0, 2, 1), vn)
+    assert _rel(s, want) < 1e-13
+
+
+def test_ones_value_is_cumsum(oracle_mod):
+    """With V = 1, every output column equals q_t . (k_1 + ... + k_t)."""
+    N, d = 180, 24
+    q = _rand((1, N, d), 1)
+    k = _rand((1, N, d), 2)
+    v = np.ones((1, N, 5))
+    o, _ = oracle_mod.recurrent(q, k, v)
+    want = np.einsum("ti,ti->t", q[0], np.cumsum(k[0], axis=0))
+    for j in range(5):
+        assert _rel(o[0, :, j], want) < 1e-13
+
+
+def test_linearity_and_causality(oracle_mod):
+    N, d = 97, 16
+    q = _rand((1, N, d), 1)
+    k = _rand((1, N, d), 2)
+    v1 = _rand((1, N, d), 3)
+    v2 = _rand((1, N, d), 4)
+    a, b = 0.75, -2.5
+    o1, _ = oracle_mod.recurrent(q, k, v1)
+    o2, _ = oracle_mod.recurrent(q, k, v2)
+    o12, _ = oracle_mod.recurrent(q, k, a * v1 + b * v2)
+    assert _rel(o12, a * o1 + b * o2) < 1e-12
+    q2 = _rand((1, N, d), 5)
+    oq, _ = oracle_mod.recurrent(q2, k, v1)
+    oqq, _ = oracle_mod.recurrent(a * q + b * q2, k, v1)
+    assert _rel(oqq, a * o1 + b * oq) < 1e-12
+    # causality: perturbing token t leaves o_{<t} untouched and changes o_t
+    t = 41
+    kp, vp = k.copy(), v1.copy()
+    kp[0, t] += 1.0
+    vp[0, t] -= 2.0
+    op, _ = oracle_mod.recurrent(q, kp, vp)
+    np.testing.assert_array_equal(op[0, :t], o1[0, :t])
+    assert np.abs(op[0, t] - o1[0, t]).max() > 1e-3
+
+
+def test_split_invariance(oracle_mod):
+    """prefill(0..n) then resume(n..N) from its state equals prefill(0..N)."""
+    q, k, v = synth.qkv((2, 500, 32), 32, "fp32", seed=8)
+    s0 = _rand((2, 32, 32), 1)
+    o, s = oracle_mod.recurrent(q, k, v, s0)
+    for n in (1, 128, 333):
+        oa, sa = oracle_mod.recurrent(q[:, :n], k[:, :n], v[:, :n], s0)
+        ob, sb = oracle_mod.recurrent(q[:, n:], k[:, n:], v[:, n:], sa)
+        assert _rel(np.concatenate([oa, ob], 1), o) < 1e-13
+        assert _rel(sb, s) < 1e-13
+
+
+def test_decode_matches_prefill(oracle_mod):
+    q, k, v = synth.qkv((3, 4, 20, 16), 16, "fp32", seed=21)
+    S0 = _rand((3, 4, 16, 16), 2)
+    o, s = oracle_mod.recurrent(q, k, v, S0)
+    S = S0.copy()
+    for t in range(20):
+        ot, S = oracle_mod.decode(q[:, :, t], k[:, :, t], v[:, :, t], S)
+        assert _rel(ot, o[:, :, t]) < 1e-13
+    assert _rel(S, s) < 1e-13
+
+
+def test_varlen_matches_loop(oracle_mod):
+    lens = [5, 0, 130, 1, 64, 77]
+    H, d = 3, 8
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    q, k, v = synth.qkv((T, H, d), d, "fp32", seed=4)
+    pool = _rand((2, H, d, d), 3)
+    idx = [1, -1, 0, -1, 1, 0]
+    o, s = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    for n, L in enumerate(lens):
+        a, b = int(cu[n]), int(cu[n + 1])
+        s0 = pool[idx[n]] if idx[n] >= 0 else None
+        qn = q[a:b].permute(1, 0, 2)
+        kn = k[a:b].permute(1, 0, 2)
+        vn = v[a:b].permute(1, 0, 2)
+        on, sn = oracle_mod.recurrent(qn, kn, vn, s0)
+        assert np.array_equal(o[a:b], on.transpose(1, 0, 2))
+        want_s = sn if L else (s0 if s0 is not None else np.zeros((H, d, d)))
+        assert np.array_equal(s[n], want_s)
+
+
+def test_empty_sequence(oracle_mod):
+    q = np.zeros((2, 0, 8))
+    s0 = _rand((2, 8, 8), 1)
+    o, s = oracle_mod.recurrent(q, q, q, s0)
+    assert o.shape == (2, 0, 8)
+    np.testing.assert_array_equal(s, s0)
+
+
+# ------------------------------------------------- planted mistakes (mutants)
+def _mutant_exclusive(q, k, v, s0):
+    """Wrong: o_t = q_t S_{t-1} (mask without the diagonal)."""
+    S = s0.copy()
+    o = np.zeros((q.shape[0], v.shape[1]))
+    for t in range(q.shape[0]):
+        o[t] = q[t] @ S
+        S = S + np.outer(k[t], v[t])
+    return o, S
+
+
+def _mutant_transposed(q, k, v, s0):
+    """Wrong: the state is read transposed, o_t = S_t q_t (needs dk == dv)."""
+    S = s0.copy()
+    o = np.zeros((q.shape[0], v.shape[1]))
+    for t in range(q.shape[0]):
+        S = S + np.outer(k[t], v[t])
+        o[t] = S @ q[t]
+    return o, S
+
+
+def _mutant_dropped_s0(q, k, v, s0):
+    """Wrong: the initial state is ignored in the outputs."""
+    o, S = _brute(q, k, v, np.zeros_like(s0))
+    return o, S + s0
+
+
+def _mutant_sign(q, k, v, s0):
+    o, S = _brute(q, k, v, s0)
+    o[1:] -= 2 * (q[1:] @ s0)
+    return o, S
+
+
+@pytest.mark.parametrize("mutant", [_mutant_exclusive, _mutant_transposed, _mutant_dropped_s0, _mutant_sign])
+def test_pins_reject_planted_mistakes(mutant):
+    """Each planted mistake fails at least one pin: the hand-worked fixture,
+    brute force with a non-zero S0, or the o_1 invariant."""
+    g = _read_golden("hand_worked_n3_d2.txt")
+    q, k, v = (g[x].reshape(3, 2) for x in ("q", "k", "v"))
+    s0 = g["B.S0"].reshape(2, 2)
+    o, s = mutant(q, k, v, s0)
+    fixture_ok = np.array_equal(o.reshape(-1), g["B.o"]) and np.array_equal(s.reshape(-1), g["B.S"])
+    qr, kr, vr, sr = _rand((6, 4), 1), _rand((6, 4), 2), _rand((6, 4), 3), _rand((4, 4), 4)
+    om, sm = mutant(qr, kr, vr, sr)
+    ob, sb = _brute(qr, kr, vr, sr)
+    brute_ok = _rel(om, ob) < 1e-12 and _rel(sm, sb) < 1e-12
+    assert not (fixture_ok and brute_ok)
