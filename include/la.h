@@ -1,0 +1,139 @@
+/*
+ * la.h — C ABI of the B200 (sm_100a) causal linear attention library.
+ *
+ * The operation (page "MiniMax-M1で理解する：大規模言語モデルのコンテキスト長
+ * 限界を突破する革新的アーキテクチャ" (zenn.dev), section "線形アテンションの
+ * 数学的基礎"), with the feature map phi = identity, no decay, no normaliser and
+ * no 1/sqrt(d) scale (the pages fix none of them):
+ *
+ *     S_t = S_{t-1} + k_t (x) v_t        (outer product; S is d_k x d_v, fp32)
+ *     o_t = q_t S_t                      (q_t a row vector; inclusive of token t)
+ *
+ * computed in tiles as Lightning Attention (page "MiniMax: «Почему M2 в итоге
+ * стала моделью с полным вниманием?» (конспект)" (ai.flicky.cc), section 1,
+ * glossary entry "Lightning Attention"): for each chunk c of C tokens,
+ *
+ *     O_c = (Q_c K_c^T ⊙ M) V_c + Q_c S_{c-1},   S_c = S_{c-1} + K_c^T V_c
+ *
+ * where M keeps s <= t (diagonal included).  The running state is the
+ * prefix-cache object of page "MiniMax: «Почему M2 …»", section 4
+ * (prefix caching and state precision): it is exported in fp32 and can be
+ * fed back to resume a sequence.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Ownership: the caller allocates and owns every buffer; the library never
+ *    allocates device memory.  All pointers are DEVICE pointers unless noted.
+ *  - Streams: work is enqueued on `stream` (NULL = the legacy default stream)
+ *    and the call returns without waiting; errors found on the host come back
+ *    as la_status, launch errors as LA_ERR_CUDA (see la_last_error()).
+ *  - Alignment: every tensor pointer must be 16-byte aligned.
+ *  - Aliasing: no input may alias an output, except the in-place state of
+ *    la_decode_step.
+ *  - Dimensions: d_k = d_v = d with d in {64, 128}.  bf16 inputs with d = 128
+ *    run on the tcgen05 tensor-core path; fp32 inputs and d = 64 run on a
+ *    CUDA-core FFMA path.  Anything else returns LA_ERR_UNSUPPORTED.
+ *  - Output dtype equals the input dtype; states are always fp32.
+ *  - Device-side waits are bounded; a wait that runs out records
+ *    LA_ERR_TIMEOUT in a device status word read by la_device_status().
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, bad cu_seqlens ... */
+    LA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, d, chunk)             */
+    LA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed             */
+    LA_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out                      */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
+
+/* Same type as cudaStream_t (an opaque CUDA stream handle). */
+typedef struct CUstream_st* la_stream_t;
+
+/* Static description of a status code. Never NULL. */
+LA_API const char* la_status_string(la_status s);
+
+/* Text of the last error raised on the calling host thread ("" if none). */
+LA_API const char* la_last_error(void);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+LA_API int la_version(void);
+
+/*
+ * Dense prefill.
+ *   q, k : [B, H, N, d]  dtype `dt`, contiguous (d fastest)
+ *   v, o : [B, H, N, d]  dtype `dt`; o is written
+ *   s0   : [B, H, d, d]  fp32 state before token 1, or NULL for zero
+ *   s_out: [B, H, d, d]  fp32 state after token N, or NULL (not written)
+ *   chunk: tile length C (0 = library choice).  Tensor-core path: 128;
+ *          FFMA path: 32 or 64 (default 64).  C does not change the result
+ *          beyond rounding.
+ *   workspace/ws_bytes: scratch of at least la_prefill_workspace_size(...)
+ *          bytes (may be NULL when that size is 0).
+ * N = 0 writes s_out = s0 (or zero).  Returns LA_OK once enqueued.
+ */
+LA_API size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt);
+LA_API la_status la_prefill(const void* q, const void* k, const void* v, void* o,
+                     const float* s0, float* s_out,
+                     int B, int H, int N, int dk, int dv, la_dtype dt, int chunk,
+                     void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
+ * Ragged (packed) prefill with prefix resume.
+ *   q, k : [T, H, d], v, o : [T, H, d]  dtype `dt` (token-major packing)
+ *   cu_seqlens: int32 device [n_seq+1]; sequence n covers tokens
+ *          [cu_seqlens[n], cu_seqlens[n+1]); cu_seqlens[0] = 0, non-decreasing,
+ *          cu_seqlens[n_seq] <= T.  Contents are a precondition; they are
+ *          checked (with a device-to-host copy and a stream sync) only when the
+ *          environment variable LA_VALIDATE=1 is set.
+ *   state_pool: fp32 [n_pool, H, d, d] or NULL; init_idx: int32 device [n_seq]
+ *          or NULL.  Sequence n starts from state_pool[init_idx[n]] when
+ *          init_idx[n] >= 0, else from zero.  (Prefix caching: a shared prompt
+ *          prefix is absorbed once and its state resumed by many sequences.)
+ *   s_out: fp32 [n_seq, H, d, d] final state per sequence, or NULL.
+ *   A sequence of length 0 writes its initial state to s_out.
+ *   workspace: at least la_prefill_varlen_workspace_size(...) bytes (device).
+ */
+LA_API size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt);
+LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o,
+                            const int32_t* cu_seqlens, int n_seq, int T,
+                            const float* state_pool, int n_pool, const int32_t* init_idx,
+                            float* s_out, int H, int dk, int dv, la_dtype dt, int chunk,
+                            void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
+ * One decode step for B*H independent states (page "MiniMax: «Почему M2 …»",
+ * section 4: a small state matrix read and written on every step).
+ *   q, k : [B, H, d], v, o : [B, H, d]  dtype `dt`
+ *   S    : [B, H, d, d] fp32, updated IN PLACE: S <- S + k (x) v, then o = q S.
+ */
+LA_API la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S,
+                         int B, int H, int dk, int dv, la_dtype dt, la_stream_t stream);
+
+/*
+ * Reads the device status word of the current device (synchronizes the
+ * device).  *out receives LA_OK or LA_ERR_TIMEOUT; clear != 0 resets it.
+ */
+LA_API la_status la_device_status(int* out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

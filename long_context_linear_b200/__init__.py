@@ -1,0 +1,175 @@
+"""Causal linear attention (Lightning Attention, phi = identity) for B200.
+
+Python binding of the C ABI in ``include/la.h``: every function below only
+checks and marshals arguments (torch tensors -> device pointers, the current
+CUDA stream) and calls the CUDA library; all computation runs in its kernels.
+
+    S_t = S_{t-1} + k_t (x) v_t,   o_t = q_t S_t
+
+(page "MiniMax-M1で理解する…" (zenn.dev), section "線形アテンションの数学的基礎";
+tiled as on page "MiniMax: «Почему M2 в итоге стала моделью с полным
+вниманием?»", section 1, glossary entry "Lightning Attention").
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+from ._abi import LAError, lib
+
+__all__ = ["prefill", "prefill_varlen", "decode_step", "device_status", "LAError", "lib",
+           "prefill_workspace_size", "prefill_varlen_workspace_size"]
+
+_DT = {torch.bfloat16: _abi.LA_BF16, torch.float32: _abi.LA_FP32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+    return _DT[t.dtype]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def prefill_workspace_size(B: int, H: int, N: int, d: int, dtype: torch.dtype) -> int:
+    return int(lib.la_prefill_workspace_size(B, H, N, d, d, _DT[dtype]))
+
+
+def prefill_varlen_workspace_size(n_seq: int, T: int, H: int, d: int, dtype: torch.dtype) -> int:
+    return int(lib.la_prefill_varlen_workspace_size(n_seq, T, H, d, d, _DT[dtype]))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torch.Tensor] = None, *,
+            chunk: int = 0, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
+            return_state: bool = True, workspace: Optional[torch.Tensor] = None
+            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Dense prefill over q, k, v of shape [B, H, N, d]; returns (O, S_N).
+
+    s0 (fp32 [B, H, d, d]) is the state before the first token (zero if None).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, q.device)
+    if q.dim() != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B, H, N, dk] and v [B, H, N, dv]")
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, q.device)
+    if s0 is not None:
+        _need(s0, "s0", torch.float32, q.device)
+        if tuple(s0.shape) != (B, H, dk, dv):
+            raise ValueError("s0 must be [B, H, dk, dv]")
+    if s_out is None and return_state:
+        s_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if s_out is not None:
+        _need(s_out, "s_out", torch.float32, q.device)
+    need = int(lib.la_prefill_workspace_size(B, H, N, dk, dv, dt))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(s0), _ptr(s_out),
+                                  B, H, N, dk, dv, dt, chunk, _ptr(workspace), ws_bytes, _stream(q.device)),
+                   "la_prefill")
+    return out, s_out
+
+
+def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                   state_pool: Optional[torch.Tensor] = None, init_idx: Optional[torch.Tensor] = None, *,
+                   chunk: int = 0, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
+                   return_state: bool = True, workspace: Optional[torch.Tensor] = None
+                   ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Packed ragged prefill: q, k [T, H, d], v [T, H, d], cu_seqlens int32 [n_seq + 1].
+
+    Sequence n starts from state_pool[init_idx[n]] when init_idx[n] >= 0.
+    Returns (O [T, H, d], S [n_seq, H, d, d]).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, q.device)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k must be [T, H, dk] and v [T, H, dv]")
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n_seq = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, q.device)
+    n_pool = 0
+    if state_pool is not None:
+        _need(state_pool, "state_pool", torch.float32, q.device)
+        n_pool = state_pool.shape[0]
+        if tuple(state_pool.shape[1:]) != (H, dk, dv):
+            raise ValueError("state_pool must be [n_pool, H, dk, dv]")
+    if init_idx is not None:
+        _need(init_idx, "init_idx", torch.int32, q.device)
+        if init_idx.numel() != n_seq:
+            raise ValueError("init_idx must have n_seq entries")
+    if s_out is None and return_state:
+        s_out = torch.empty((max(n_seq, 0), H, dk, dv), dtype=torch.float32, device=q.device)
+    if s_out is not None:
+        _need(s_out, "s_out", torch.float32, q.device)
+    need = int(lib.la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq, T,
+                                         _ptr(state_pool), n_pool, _ptr(init_idx), _ptr(s_out), H, dk, dv, dt,
+                                         chunk, _ptr(workspace), ws_bytes, _stream(q.device)),
+                   "la_prefill_varlen")
+    return out, s_out
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token per (batch, head): S <- S + k (x) v in place, returns o = q S.
+
+    q, k, v: [B, H, d]; S: fp32 [B, H, d, d].
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, q.device)
+    _need(S, "S", torch.float32, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k must be [B, H, dk] and v [B, H, dv]")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(S.shape) != (B, H, dk, dv):
+        raise ValueError("S must be [B, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, q.device)
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, dk, dv,
+                                      _dtype_code(q), _stream(q.device)), "la_decode_step")
+    return out
+
+
+def device_status(clear: bool = True) -> int:
+    """Device status word (0 = ok, 4 = a bounded device wait timed out). Synchronizes."""
+    import ctypes
+    v = ctypes.c_int(0)
+    _abi.check(lib.la_device_status(ctypes.byref(v), 1 if clear else 0), "la_device_status")
+    return int(v.value)

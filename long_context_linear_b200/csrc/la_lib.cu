@@ -1,0 +1,406 @@
+// C ABI of the causal linear attention library (see include/la.h): argument
+// validation, launch planning, TMA descriptor encoding and kernel launches.
+// The library allocates no device memory; TMA descriptors are encoded per call
+// on the host and passed by value as kernel parameters.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "la.h"
+#include "sm100.cuh"
+#include "prefill_tc.cuh"
+#include "prefill_simt.cuh"
+#include "decode.cuh"
+#include "varlen_order.cuh"
+
+namespace lcl {
+
+// Device status word: 0, or LA_ERR_TIMEOUT after a bounded wait ran out.
+__device__ int g_status_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+thread_local char g_last_error[512] = "";
+
+la_status fail(la_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+la_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(LA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+    int sms = 0;
+    int* status = nullptr;       // device address of g_status_word
+    bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+template <typename T>
+cudaError_t set_simt_attrs() {
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(simt::prefill_simt_kernel<T, 128, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  simt::smem_bytes<128, 64>())) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(simt::prefill_simt_kernel<T, 128, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  simt::smem_bytes<128, 32>())) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(simt::prefill_simt_kernel<T, 64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  simt::smem_bytes<64, 64>())) != cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(simt::prefill_simt_kernel<T, 64, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                simt::smem_bytes<64, 32>());
+}
+
+la_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.attrs_set) {
+        int major = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        if (major != 10) return fail(LA_ERR_UNSUPPORTED, "device %d is sm_%d x, this build targets sm_100a", dev, major);
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress");
+        if ((e = cudaFuncSetAttribute(tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      tc::SMEM_BYTES)) != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
+        if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
+        d.attrs_set = true;
+    }
+    *out = &d;
+    return LA_OK;
+}
+
+la_status encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    *out = g_encode;
+    return LA_OK;
+}
+
+// 3-D bf16 tensor map with a 64-element (128-byte) inner box and 128B swizzle.
+la_status make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+                   uint64_t stride2_bytes, uint32_t b1, uint32_t b2) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    la_status s = encoder(&enc);
+    if (s != LA_OK) return s;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {64, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LA_OK;
+}
+
+bool env_validate() {
+    const char* v = getenv("LA_VALIDATE");
+    return v && v[0] == '1';
+}
+
+la_status check_dims(int dk, int dv, la_dtype dt) {
+    if (dt != LA_BF16 && dt != LA_FP32) return fail(LA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (dk <= 0 || dv <= 0) return fail(LA_ERR_INVALID_ARG, "dk=%d dv=%d must be positive", dk, dv);
+    if (dk != dv || (dk != 64 && dk != 128))
+        return fail(LA_ERR_UNSUPPORTED, "only dk = dv in {64, 128} is supported (got %d, %d)", dk, dv);
+    return LA_OK;
+}
+
+bool use_tensor_cores(int d, la_dtype dt) { return dt == LA_BF16 && d == 128; }
+
+constexpr int kSimtDefaultChunk = 64;
+
+la_status check_chunk(int chunk, bool tcpath) {
+    if (chunk == 0) return LA_OK;
+    if (tcpath && chunk == tc::C) return LA_OK;
+    if (!tcpath && (chunk == 32 || chunk == 64)) return LA_OK;
+    return fail(LA_ERR_UNSUPPORTED, "chunk %d is not available on this path (%s)", chunk,
+                tcpath ? "tensor-core path: 0 or 128" : "FFMA path: 0, 32 or 64");
+}
+
+la_status after_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return LA_OK;
+}
+
+template <typename T, int D>
+void launch_simt_d(int cs, int grid, const void* q, const void* k, const void* v, void* o, const simt::Params& sp,
+                   cudaStream_t st) {
+    if (cs == 32)
+        simt::prefill_simt_kernel<T, D, 32><<<grid, simt::NUM_THREADS, simt::smem_bytes<D, 32>(), st>>>(
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, sp);
+    else
+        simt::prefill_simt_kernel<T, D, 64><<<grid, simt::NUM_THREADS, simt::smem_bytes<D, 64>(), st>>>(
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, sp);
+}
+
+template <typename T>
+la_status launch_simt(int d, int chunk, int grid, const void* q, const void* k, const void* v, void* o,
+                      const simt::Params& sp, cudaStream_t st) {
+    if (grid == 0) return LA_OK;
+    const int cs = chunk ? chunk : kSimtDefaultChunk;
+    if (d == 128) launch_simt_d<T, 128>(cs, grid, q, k, v, o, sp, st);
+    else launch_simt_d<T, 64>(cs, grid, q, k, v, o, sp, st);
+    return after_launch("prefill_simt launch");
+}
+
+}  // namespace
+}  // namespace lcl
+
+using namespace lcl;
+
+extern "C" {
+
+const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: unsupported configuration";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA error";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: a device-side wait timed out";
+    }
+    return "unknown la_status";
+}
+
+const char* la_last_error(void) { return g_last_error; }
+
+int la_version(void) { return 100; }
+
+size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt) {
+    (void)B; (void)H; (void)N; (void)dk; (void)dv; (void)dt;
+    return 0;
+}
+
+la_status la_prefill(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
+                     int H, int N, int dk, int dv, la_dtype dt, int chunk, void* workspace, size_t ws_bytes,
+                     la_stream_t stream) {
+    (void)workspace; (void)ws_bytes;
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || N < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d N=%d", B, H, N);
+    const long U = (long)B * H;
+    if (U > (1L << 30) || (long)N * U > (1L << 40)) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (U == 0) return LA_OK;
+    if (N > 0 && (!q || !k || !v || !o)) return fail(LA_ERR_INVALID_ARG, "q, k, v, o must be non-null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(s0) || !aligned16(s_out))
+        return fail(LA_ERR_INVALID_ARG, "all pointers must be 16-byte aligned");
+    const bool tcpath = use_tensor_cores(dk, dt);
+    if ((s = check_chunk(chunk, tcpath)) != LA_OK) return s;
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    if (!tcpath) {
+        simt::Params sp{};
+        sp.mode = 0; sp.N = N; sp.s0 = s0; sp.s_out = s_out;
+        if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)U, q, k, v, o, sp, st);
+        return launch_simt<__nv_bfloat16>(dk, chunk, (int)U, q, k, v, o, sp, st);
+    }
+
+    tc::Params p{};
+    p.mode = 0;
+    p.n_vs = dv / tc::DVS;
+    p.n_items = (int)(U * p.n_vs);
+    p.H = H;
+    p.N = N;
+    p.dv = dv;
+    p.s0 = s0;
+    p.s_out = s_out;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.status = di->status;
+    if (N == 0 && !s_out) return LA_OK;
+    // With N = 0 no tile is ever copied; the maps then only need a valid base.
+    const void* bq = N > 0 ? q : s_out;
+    const void* bk = N > 0 ? k : s_out;
+    const void* bv = N > 0 ? v : s_out;
+    const void* bo = N > 0 ? o : s_out;
+    CUtensorMap mq, mk, mv, mo;
+    const uint64_t row = (uint64_t)dk * 2;
+    const uint64_t Nm = N > 0 ? (uint64_t)N : 1;
+    const uint64_t unit = Nm * row;
+    if ((s = make_map(&mq, bq, dk, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mk, bk, dk, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mv, bv, dv, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mo, bo, dv, Nm, U, row, unit, 32, 1)) != LA_OK) return s;
+    const int grid = std::min(p.n_items, di->sms);
+    tc::prefill_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    return after_launch("prefill_tc launch");
+}
+
+size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt) {
+    (void)T; (void)H; (void)dk; (void)dv; (void)dt;
+    if (n_seq <= 0) return 0;
+    return ((size_t)n_seq * sizeof(int) + 255) & ~(size_t)255;
+}
+
+la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                            int n_seq, int T, const float* state_pool, int n_pool, const int32_t* init_idx,
+                            float* s_out, int H, int dk, int dv, la_dtype dt, int chunk, void* workspace,
+                            size_t ws_bytes, la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (n_seq < 0 || T < 0 || H < 0 || n_pool < 0)
+        return fail(LA_ERR_INVALID_ARG, "negative size n_seq=%d T=%d H=%d n_pool=%d", n_seq, T, H, n_pool);
+    if (n_seq == 0 || H == 0) return LA_OK;
+    if (!cu_seqlens) return fail(LA_ERR_INVALID_ARG, "cu_seqlens must be non-null");
+    if (T > 0 && (!q || !k || !v || !o)) return fail(LA_ERR_INVALID_ARG, "q, k, v, o must be non-null");
+    if (init_idx && (!state_pool || n_pool == 0))
+        return fail(LA_ERR_INVALID_ARG, "init_idx given without a state pool");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state_pool) ||
+        !aligned16(s_out) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(init_idx) & 3u))
+        return fail(LA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned, index arrays 4-byte aligned");
+    if ((long)T * H > (1L << 40) || (long)n_seq * H > (1L << 30)) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    const bool tcpath = use_tensor_cores(dk, dt);
+    if ((s = check_chunk(chunk, tcpath)) != LA_OK) return s;
+    const size_t need = la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt);
+    if (tcpath && (ws_bytes < need || !workspace || !aligned16(workspace)))
+        return fail(LA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu", need, ws_bytes);
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    if (env_validate()) {
+        std::vector<int32_t> cu(n_seq + 1), idx;
+        cudaError_t e = cudaMemcpyAsync(cu.data(), cu_seqlens, sizeof(int32_t) * (n_seq + 1), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess && init_idx) {
+            idx.resize(n_seq);
+            e = cudaMemcpyAsync(idx.data(), init_idx, sizeof(int32_t) * n_seq, cudaMemcpyDeviceToHost, st);
+        }
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "LA_VALIDATE copy of cu_seqlens");
+        if (cu[0] != 0) return fail(LA_ERR_INVALID_ARG, "cu_seqlens[0] = %d, expected 0", cu[0]);
+        for (int n = 0; n < n_seq; ++n)
+            if (cu[n + 1] < cu[n]) return fail(LA_ERR_INVALID_ARG, "cu_seqlens decreases at %d", n);
+        if (cu[n_seq] > T) return fail(LA_ERR_INVALID_ARG, "cu_seqlens[n_seq] = %d exceeds T = %d", cu[n_seq], T);
+        for (size_t n = 0; n < idx.size(); ++n)
+            if (idx[n] < -1 || idx[n] >= n_pool)
+                return fail(LA_ERR_INVALID_ARG, "init_idx[%zu] = %d outside [-1, %d)", n, idx[n], n_pool);
+    }
+
+    if (!tcpath) {
+        simt::Params sp{};
+        sp.mode = 1; sp.H = H; sp.cu_seqlens = cu_seqlens; sp.pool = state_pool; sp.init_idx = init_idx;
+        sp.s_out = s_out;
+        const long grid = (long)n_seq * H;
+        if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)grid, q, k, v, o, sp, st);
+        return launch_simt<__nv_bfloat16>(dk, chunk, (int)grid, q, k, v, o, sp, st);
+    }
+
+    int* order = reinterpret_cast<int*>(workspace);
+    vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
+    if ((s = after_launch("varlen order launch")) != LA_OK) return s;
+
+    tc::Params p{};
+    p.mode = 1;
+    p.n_vs = dv / tc::DVS;
+    p.n_items = (int)((long)n_seq * H * p.n_vs);
+    p.H = H;
+    p.dv = dv;
+    p.cu_seqlens = cu_seqlens;
+    p.order = order;
+    p.pool = state_pool;
+    p.init_idx = init_idx;
+    p.s_out = s_out;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.status = di->status;
+    CUtensorMap mq, mk, mv, mo;
+    const uint64_t Tm = T > 0 ? (uint64_t)T : 1;
+    const uint64_t head = (uint64_t)dk * 2, tok = (uint64_t)H * dk * 2;
+    const void* any = q ? q : (const void*)order;
+    if ((s = make_map(&mq, q ? q : any, dk, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
+    if ((s = make_map(&mk, k ? k : any, dk, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
+    if ((s = make_map(&mv, v ? v : any, dv, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
+    if ((s = make_map(&mo, o ? o : any, dv, H, Tm, head, tok, 1, 32)) != LA_OK) return s;
+    const int grid = std::min(p.n_items, di->sms);
+    tc::prefill_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    return after_launch("prefill_tc (varlen) launch");
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S, int B, int H, int dk,
+                         int dv, la_dtype dt, la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
+    const long U = (long)B * H;
+    if (U == 0) return LA_OK;
+    if (U > (1L << 31) - 1) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (!q || !k || !v || !o || !S) return fail(LA_ERR_INVALID_ARG, "q, k, v, o, S must be non-null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S))
+        return fail(LA_ERR_INVALID_ARG, "all pointers must be 16-byte aligned");
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int grid = (int)U;
+    if (dt == LA_BF16) {
+        using T = __nv_bfloat16;
+        if (dk == 128) dec::decode_step_kernel<T, 128><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+        else dec::decode_step_kernel<T, 64><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+    } else {
+        using T = float;
+        if (dk == 128) dec::decode_step_kernel<T, 128><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+        else dec::decode_step_kernel<T, 64><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+    }
+    return after_launch("decode_step launch");
+}
+
+la_status la_device_status(int* out, int clear) {
+    g_last_error[0] = 0;
+    if (!out) return fail(LA_ERR_INVALID_ARG, "out must be non-null");
+    DeviceInfo* di;
+    la_status s = device_info(&di);
+    if (s != LA_OK) return s;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    if ((e = cudaMemcpy(&v, di->status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "status read");
+    if (clear && (e = cudaMemset(di->status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
+    *out = v;
+    return LA_OK;
+}
+
+}  // extern "C"
