@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the causal linear attention hot path on B200.
+
+Headline (one JSON line on rank 0): long prefill, B=1, H=64, N=131072, d=128,
+bf16 inputs, fp32 state, zero initial state, returning O and the final S.
+One step = one la_prefill call over that batch; value = prefill tokens/s
+(B*N tokens per step, all ranks summed).  Inputs (6 GiB) are larger than L2,
+so no flush is needed between steps.
+
+Also reported in the same line (same timing rules): the batched decode step
+(B=256, H=64, d=128, 1024 consecutive steps, achieved HBM GB/s), the ragged
+varlen prefill with prefix resume (64 sequences, lengths ~U[1K,32K], H=32)
+and the B=4, H=32, N=8192 prefill.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+headline workload instead (rank 0 only).
+
+Multi-GPU: every rank runs the same per-GPU workload on its own inputs
+(weak scaling; the units are independent, there is no data-path collective);
+times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+HEADLINE = dict(B=1, H=64, N=131072, d=128)
+DECODE = dict(B=256, H=64, d=128, steps=1024, L_lo=1024, L_hi=65536)
+VARLEN = dict(n_seq=64, lo=1024, hi=32768, H=32, d=128, n_resume=32, prefix=4096)
+PREFILL8K = dict(B=4, H=32, N=8192, d=128)
+METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples for one GPU while a region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            self.bus = "%04x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            ids = [x.strip() for x in vis.split(",")] if vis else None
+            self.bus = ids[device_index] if ids and device_index < len(ids) else str(device_index)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 8:
+                rows.append(parts)
+        if not rows:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"], samples=0)
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        power = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        # samples under load: SM clock at least half of its max
+        load = [s for s in sm if mx and s >= 0.5 * max(mx)] or sm
+        return dict(sm_mhz=statistics.median(load) if load else None, sm_max_mhz=max(mx) if mx else None,
+                    reasons=reasons, samples=len(rows), power_w_max=max(power) if power else None)
+
+
+def flops_rec(tokens_heads: float, d: int) -> float:
+    """Algorithmic FLOPs of the recurrence: d*d multiply-adds to update S and d*d
+    to form o, per token and head (4 d^2)."""
+    return 4.0 * d * d * tokens_heads
+
+
+def flops_issued(tokens_heads: float, d: int, C: int = 128, slice_w: int = 64) -> float:
+    """FLOPs the tensor cores execute: per 64-wide value slice, Q K^T (2 C d),
+    P V (2 C w), Q S_hi + Q S_lo (4 d w) and K^T V (2 d w) per token."""
+    n_vs = d // slice_w
+    return tokens_heads * n_vs * (2 * C * d + 2 * C * slice_w + 4 * d * slice_w + 2 * d * slice_w)
+
+
+def prefill_bytes(B, H, N, d) -> float:
+    """Algorithmic HBM bytes: read Q, K, V, write O (bf16), write S (fp32)."""
+    return 4.0 * B * H * N * d * 2 + B * H * d * d * 4
+
+
+# ----------------------------------------------------------------- our arm
+def timed_launches(fn, steps: int, warmup: int, dist: Dist, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = t_all0.elapsed_time(t_all1)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, per_launch
+
+
+def run_headline(args, dist: Dist, pk, sampler: ClockSampler):
+    import long_context_linear_b200 as la
+    import synth
+    B, H, N, d = HEADLINE["B"], args.heads, args.seq, HEADLINE["d"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=3 + 1000 * dist.rank, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        la.prefill(q, k, v, None, out=o, s_out=s)
+
+    sampler.start()
+    total_ms, per_launch = timed_launches(step, args.steps, args.warmup, dist, stream)
+    clocks = sampler.stop()
+    total_ms = dist.max(total_ms)
+    launch_ms = dist.max(statistics.fmean(per_launch))
+    ms_step = total_ms / args.steps
+    tokens = B * N * dist.world
+    value = tokens / (ms_step / 1e3)
+    if (H, N) != (HEADLINE["H"], HEADLINE["N"]):
+        print(f"note: headline workload overridden to H={H} N={N}", file=sys.stderr)
+    th = B * H * N
+    bytes_launch = prefill_bytes(B, H, N, d)
+    achieved_gbs = bytes_launch / (launch_ms / 1e3) / 1e9
+    f_rec = flops_rec(th, d) / (launch_ms / 1e3) / 1e12
+    f_iss = flops_issued(th, d) / (launch_ms / 1e3) / 1e12
+
+    # end to end through the public call with host buffers (pinned), copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        sh = torch.empty(s.shape, dtype=s.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            la.prefill(qd, kd, vd, None, out=o, s_out=s)
+            oh.copy_(o, non_blocking=True)
+            sh.copy_(s, non_blocking=True)
+
+        n_e2e = min(args.e2e_steps, args.steps)
+        e_total, _ = timed_launches(e2e_step, n_e2e, 1, dist, stream)
+        e_total = dist.max(e_total)
+        e2e = dict(value=tokens / (e_total / n_e2e / 1e3), unit="tokens/s",
+                   h2d_bytes_per_step=3 * q.numel() * q.element_size(),
+                   d2h_bytes_per_step=o.numel() * o.element_size() + s.numel() * s.element_size(),
+                   steps=n_e2e)
+        del qh, kh, vh, oh, sh, qd, kd, vd
+    sample = dict(q=q[0, :2, :256].float().cpu(), k=k[0, :2, :256].float().cpu(), v=v[0, :2, :256].float().cpu())
+    del q, k, v, o, s
+    torch.cuda.empty_cache()
+    res = dict(value=value, ms_per_step=ms_step, launch_ms=launch_ms, achieved_gbs=achieved_gbs,
+               bytes_launch=bytes_launch, tflops_rec=f_rec, tflops_issued=f_iss, clocks=clocks, e2e=e2e,
+               launches=args.steps)
+    return res, sample
+
+
+def run_decode(args, dist: Dist, pk):
+    import long_context_linear_b200 as la
+    import synth
+    c = DECODE
+    B, H, d, steps = c["B"], c["H"], c["d"], c["steps"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    U = B * H
+    L_seq = synth.lengths(B, c["L_lo"], c["L_hi"], seed=41 + dist.rank)
+    L = [L_seq[u // H] for u in range(U)]
+    S = torch.empty(U, d, d, dtype=torch.float32, device=dev)
+    grp = 2048
+    for u0 in range(0, U, grp):
+        S[u0:u0 + grp] = synth.outer_product_state(min(grp, U - u0), d, d, L[u0:u0 + grp], seed=7 + u0, device=dev)
+    S = S.view(B, H, d, d)
+    qs, ks, vs = synth.qkv((steps, B, H, d), d, "bf16", seed=43 + dist.rank, device=dev)
+    os_ = torch.empty_like(vs)
+    stream = torch.cuda.current_stream(dev)
+    it = [0]
+
+    def step():
+        t = it[0] % steps
+        la.decode_step(qs[t], ks[t], vs[t], S, out=os_[t])
+        it[0] += 1
+
+    # warm-up, then time `steps` consecutive decode steps
+    total_ms, per = timed_launches(step, steps, max(3, args.warmup), dist, stream)
+    total_ms = dist.max(total_ms)
+    ms_step = total_ms / steps
+    bytes_step = 2.0 * U * d * d * 4 + 4.0 * U * d * 2
+    gbs = bytes_step / (ms_step / 1e3) / 1e9
+    del S, qs, ks, vs, os_
+    torch.cuda.empty_cache()
+    return dict(workload="decode B=256 H=64 d=128 bf16 q/k/v, fp32 state, 1024 consecutive steps",
+                hbm_gbs=gbs, peak_gbs=pk["hbm"], frac=gbs / pk["hbm"], ms_per_step=ms_step,
+                bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
+
+
+def run_varlen(args, dist: Dist, pk):
+    import long_context_linear_b200 as la
+    import synth
+    c = VARLEN
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lens = synth.lengths(c["n_seq"], c["lo"], c["hi"], seed=51 + dist.rank)
+    cu = synth.cu_seqlens(lens).to(dev)
+    T, H, d = int(cu[-1]), c["H"], c["d"]
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=53 + dist.rank, device=dev)
+    resumed = synth.choose(c["n_seq"], c["n_resume"], seed=55)
+    pool = synth.outer_product_state(c["n_resume"] * H, d, d, [c["prefix"]] * (c["n_resume"] * H), seed=57,
+                                     device=dev).view(c["n_resume"], H, d, d)
+    idx = torch.full((c["n_seq"],), -1, dtype=torch.int32)
+    for j, n in enumerate(resumed):
+        idx[n] = j
+    idx = idx.to(dev)
+    o = torch.empty_like(v)
+    s = torch.empty(c["n_seq"], H, d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(la.prefill_varlen_workspace_size(c["n_seq"], T, H, d, torch.bfloat16), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        la.prefill_varlen(q, k, v, cu, pool, idx, out=o, s_out=s, workspace=ws)
+
+    n = max(3, min(args.steps, 20))
+    total_ms, per = timed_launches(step, n, max(3, args.warmup), dist, stream)
+    total_ms = dist.max(total_ms)
+    ms_step = total_ms / n
+    byts = 4.0 * T * H * d * 2 + c["n_seq"] * H * d * d * 4 + c["n_resume"] * H * d * d * 4
+    gbs = byts / (ms_step / 1e3) / 1e9
+    del q, k, v, o, s, pool
+    torch.cuda.empty_cache()
+    return dict(workload="varlen 64 seqs len~U[1K,32K] (T=%d), H=32, d=128, bf16, 32 resumed from fp32 states" % T,
+                tokens_per_s=T * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
+                frac=gbs / pk["hbm"], tflops_rec=flops_rec(T * H, d) / (ms_step / 1e3) / 1e12, steps=n)
+
+
+def run_prefill8k(args, dist: Dist, pk):
+    import long_context_linear_b200 as la
+    import synth
+    c = PREFILL8K
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=61 + dist.rank, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = max(10, min(args.steps, 200))
+    total_ms, per = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s), n, max(3, args.warmup),
+                                   dist, stream)
+    total_ms = dist.max(total_ms)
+    ms_step = total_ms / n
+    byts = prefill_bytes(B, H, N, d)
+    gbs = byts / (ms_step / 1e3) / 1e9
+    del q, k, v, o, s
+    torch.cuda.empty_cache()
+    return dict(workload="prefill B=4 H=32 N=8192 d=128 bf16", tokens_per_s=B * N * dist.world / (ms_step / 1e3),
+                ms_per_step=ms_step, hbm_gbs=gbs, frac=gbs / pk["hbm"],
+                tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
+                l2="inputs (1 GiB) larger than L2")
+
+
+# ----------------------------------------------------------------- oracle arm
+def oracle_sample_plan(budget_s: float):
+    """Heads x tokens of the headline workload the oracle processes in about
+    ``budget_s`` seconds on this host's cores."""
+    import oracle
+    import synth
+    oracle.build()
+    threads = oracle.num_threads()
+    heads = max(1, min(threads, HEADLINE["H"]))
+    q, k, v = synth.dense(1, 1, 2048, HEADLINE["d"], "bf16", seed=0)
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v)
+    per_token = (time.perf_counter() - t0) / 2048  # one thread, one head
+    tokens = int(budget_s / per_token)
+    tokens = max(256, min(HEADLINE["N"], tokens))
+    return threads, heads, tokens
+
+
+def time_oracle(heads, tokens, steps, warmup, seed=3):
+    import oracle
+    import synth
+    q, k, v = synth.dense(1, heads, tokens, HEADLINE["d"], "bf16", seed=seed)
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    for _ in range(warmup):
+        oracle.recurrent(qd, kd, vd)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.recurrent(qd, kd, vd)
+    dt = (time.perf_counter() - t0) / steps
+    equiv_tokens = heads * tokens / HEADLINE["H"]  # headline tokens carry 64 heads each
+    return equiv_tokens / dt, dt
+
+
+def cpu_baseline_line(budget_s=12.0):
+    threads, heads, tokens = oracle_sample_plan(budget_s)
+    value, dt = time_oracle(heads, tokens, 1, 0)
+    return dict(value=value, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"fp64 recurrence on {heads} of 64 heads x first {tokens} tokens of the B=1 H=64 "
+                       f"N=131072 d=128 workload ({dt:.1f} s); value in headline tokens (64 heads each)")
+
+
+def reference_arm(args, dist: Dist):
+    if dist.rank != 0:
+        return 0
+    budget = max(0.2, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    threads, heads, tokens = oracle_sample_plan(budget)
+    value, dt = time_oracle(heads, tokens, args.steps, args.warmup)
+    sample = (f"fp64 oracle recurrence on {heads} of 64 heads x first {tokens} tokens of the headline workload "
+              f"per step; value in headline tokens (64 heads each)")
+    line = dict(impl="reference", metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=dt * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic",
+                config=dict(workload="prefill B=1 H=64 N=131072 d=128 (bf16 inputs widened to fp64)",
+                            global_batch=1, seq_len=HEADLINE["N"], heads=64, head_dim=128),
+                cpu_baseline=dict(value=value, unit="tokens/s", cores=threads, kind="oracle", sample=sample),
+                e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+                gpu_launches=0)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-extras", action="store_true", help="headline only (skip decode/varlen/8K)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=HEADLINE["H"], help="headline heads (smaller for profiling)")
+    ap.add_argument("--seq", type=int, default=HEADLINE["N"], help="headline tokens (smaller for profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    dist = Dist()
+    if args.impl == "reference":
+        return reference_arm(args, dist)
+
+    torch.cuda.set_device(dist.local)
+    dist.init("nccl")
+    pk = peaks()
+    sampler = ClockSampler(dist.local)
+    head, _ = run_headline(args, dist, pk, sampler)
+    extras = {}
+    if not args.no_extras:
+        extras["decode"] = run_decode(args, dist, pk)
+        extras["varlen"] = run_varlen(args, dist, pk)
+        extras["prefill_8k"] = run_prefill8k(args, dist, pk)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_line()
+    if dist.rank == 0:
+        d = HEADLINE["d"]
+        peak_note = "of measured" if pk["source"] == "measured" else "of fallback"
+        line = dict(
+            metric=METRIC, value=head["value"], unit="tokens/s", n_gpus=dist.world, steps=args.steps,
+            warmup=args.warmup, ms_per_step=head["ms_per_step"], higher_is_better=True, scaling="weak",
+            vs_baseline=None, dtype="bf16", data="synthetic (seeded N(0,1)/sqrt(d) q,k and N(0,1) v)",
+            config=dict(workload=f"long prefill B=1 H={args.heads} N={args.seq} d=128, bf16 in, fp32 state, "
+                                 "zero initial state, returns O and final S", global_batch=dist.world,
+                        seq_len=args.seq, heads=args.heads, head_dim=d, chunk=128,
+                        parallelism=f"replicas x{dist.world}",
+                        l2="inputs larger than L2, no flush" if 3 * args.heads * args.seq * d * 2 > 126e6
+                        else "inputs fit in L2 (profiling case)"),
+            roofline=dict(bound="hbm", achieved=head["achieved_gbs"], peak=pk["hbm"], unit="GB/s",
+                          frac=head["achieved_gbs"] / pk["hbm"], traffic=None, peak_source=peak_note,
+                          algorithmic_bytes_per_launch=head["bytes_launch"], launch_ms=head["launch_ms"]),
+            tensor=dict(tflops_rec=head["tflops_rec"], tflops_issued=head["tflops_issued"],
+                        frac_rec=head["tflops_rec"] / pk["bf16"], frac_issued=head["tflops_issued"] / pk["bf16"],
+                        peak_tflops=pk["bf16"], peak_source=peak_note),
+            e2e=head["e2e"], gpu_launches=head["launches"], clocks=head["clocks"], cpu_baseline=cpu,
+            extras=extras)
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -9,9 +9,10 @@
 //
 //   P_c   = Q_c K_c^T                      tcgen05, fp32 accumulator in TMEM
 //   P_c  <- P_c ⊙ M  (keep s <= t), bf16   mask warps, written back into TMEM
-//   O_c   = P_c V_c                        tcgen05 with A = P_c read from TMEM
-//   O_c  += Q_c S_hi + Q_c S_lo            S_{c-1} split into two bf16 terms
+//   [O|O']= Q_c [S_hi | S_lo]              one N=128 product; S_{c-1} split
+//                                          into two bf16 terms, summed on output
 //   dS_c  = K_c^T V_c                      tcgen05 (K, V read MN-major)
+//   O    += P_c V_c                        tcgen05 with A = P_c read from TMEM
 //   S_c   = S_{c-1} + dS_c                 fp32, in the state warps' registers
 //
 // Work item = (sequence or batch*head unit, head, 64-wide slice of d_v).  One
@@ -19,11 +20,16 @@
 // fp32 registers of four "state" warps; the tensor cores only ever see it as
 // S_hi = bf16(S), S_lo = bf16(S - S_hi), so the Q S product keeps ~16 bits of
 // the fp32 state.  Warp roles (14 warps):
-//   w0 lane 0 : TMA producer (Q, K, V chunk tiles, 128B-swizzled, 2 stages)
+//   w0 lane 0 : TMA producer (Q,K tiles in 2 slots, V tiles in 3 slots,
+//               128B-swizzled; L2 prefetch a few chunks ahead)
 //   w1        : TMEM allocation; lane 0 issues every tcgen05.mma
 //   w2..w5    : mask warps   (P: TMEM -> regs -> causal mask -> bf16 -> TMEM)
 //   w6..w9    : state warps  (dS: TMEM -> regs, S += dS, S_hi/S_lo -> smem)
-//   w10..w13  : output warps (O: TMEM -> regs -> bf16 -> smem -> TMA store)
+//   w10..w13  : output warps (O + O': TMEM -> regs -> bf16 -> smem -> TMA store)
+// The issue order per chunk (P, dS, Q S, P V) lets the tensor cores run dS and
+// Q S while the mask warps work on P, and gives the state warps Q S, P V and
+// the next chunk's P and dS to fold dS_c into S before it is needed.  Q/K
+// slots are released after Q S, V slots after P V.
 // Every wait is bounded (see mbar_wait); a timeout stops the CTA cleanly.
 #pragma once
 #include "sm100.cuh"
@@ -34,22 +40,40 @@ namespace tc {
 constexpr int C = 128;         // chunk length (tokens)
 constexpr int DK = 128;        // key dim
 constexpr int DVS = 64;        // value columns per CTA
-constexpr int STAGES = 2;
+constexpr int QK_SLOTS = 2;    // Q,K chunk tiles in flight (held until Q S)
+constexpr int V_SLOTS = 3;     // V chunk tiles in flight (held until P V)
+constexpr int PREFETCH = 3;    // chunks brought into L2 ahead of their load
 constexpr int PANEL = 128 * 128;  // one 128-row x 128-byte swizzled panel
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = 2 * PANEL;
-constexpr int OFF_V = 4 * PANEL;
-constexpr int STAGE_BYTES = 5 * PANEL;
-constexpr int OFF_SHI = STAGES * STAGE_BYTES;
+constexpr int QK_BYTES = 4 * PANEL;                   // Q (2 panels) + K (2 panels)
+constexpr int OFF_QK = 0;                             // QK_SLOTS x [Q0 Q1 K0 K1]
+constexpr int OFF_V = OFF_QK + QK_SLOTS * QK_BYTES;   // V_SLOTS x [V]
+constexpr int OFF_SHI = OFF_V + V_SLOTS * PANEL;      // S_hi panel, S_lo panel right after
 constexpr int OFF_SLO = OFF_SHI + PANEL;
-constexpr int OFF_OST = OFF_SLO + PANEL;   // 2 output staging panels
-constexpr int OFF_BAR = OFF_OST + 2 * PANEL;
+constexpr int OFF_OST = OFF_SLO + PANEL;              // output staging panel
+constexpr int OFF_BAR = OFF_OST + PANEL;
+// mbarrier slots (8 bytes each) at OFF_BAR, then the TMEM base and the abort flag
+constexpr int BAR_QK_FULL = 0;
+constexpr int BAR_QK_EMPTY = BAR_QK_FULL + QK_SLOTS;
+constexpr int BAR_V_FULL = BAR_QK_EMPTY + QK_SLOTS;
+constexpr int BAR_V_EMPTY = BAR_V_FULL + V_SLOTS;
+constexpr int BAR_P_FULL = BAR_V_EMPTY + V_SLOTS;
+constexpr int BAR_P_READY = BAR_P_FULL + 1;
+constexpr int BAR_DS_FULL = BAR_P_READY + 1;
+constexpr int BAR_DS_EMPTY = BAR_DS_FULL + 2;
+constexpr int BAR_O_FULL = BAR_DS_EMPTY + 2;
+constexpr int BAR_O_EMPTY = BAR_O_FULL + 2;
+constexpr int BAR_S_FULL = BAR_O_EMPTY + 2;
+constexpr int BAR_S_EMPTY = BAR_S_FULL + 1;
+constexpr int BAR_DRAIN = BAR_S_EMPTY + 1;
+constexpr int BAR_COUNT = BAR_DRAIN + 1;
 constexpr int BAR_BYTES = 256;
+static_assert((BAR_COUNT + 2) * 8 <= BAR_BYTES, "barrier area too small");
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB per-block shared memory limit");
 constexpr int NUM_THREADS = 448;
 
-constexpr uint32_t TM_P = 0;     // 2 buffers x 128 columns
-constexpr uint32_t TM_O = 256;   // 2 buffers x 64 columns
+constexpr uint32_t TM_P = 0;     // 128 columns: P (fp32), then bf16 P in columns 0..63
+constexpr uint32_t TM_O = 128;   // 2 buffers x 128 columns: [Q S_hi + P V | Q S_lo]
 constexpr uint32_t TM_DS = 384;  // 2 buffers x 64 columns
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -133,19 +157,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* full = bars + 0;      // [2] TMA -> MMA
-    uint64_t* empty = bars + 2;     // [2] MMA -> TMA
-    uint64_t* p_full = bars + 4;    // [2] MMA -> mask
-    uint64_t* p_ready = bars + 6;   // [2] mask -> MMA
-    uint64_t* ds_full = bars + 8;   // [2] MMA -> state
-    uint64_t* ds_empty = bars + 10; // [2] state -> MMA
-    uint64_t* o_full = bars + 12;   // [2] MMA -> output
-    uint64_t* o_empty = bars + 14;  // [2] output -> MMA
-    uint64_t* s_full = bars + 16;   // state -> MMA (S_hi/S_lo written)
-    uint64_t* s_empty = bars + 17;  // MMA -> state (Q S products done)
-    uint64_t* drain = bars + 18;    // MMA drain on exit
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 19);
-    volatile int* abort = reinterpret_cast<volatile int*>(bars + 20);
+    uint64_t* qk_full = bars + BAR_QK_FULL;    // [QK_SLOTS] TMA -> MMA
+    uint64_t* qk_empty = bars + BAR_QK_EMPTY;  // [QK_SLOTS] MMA -> TMA (after Q S)
+    uint64_t* v_full = bars + BAR_V_FULL;      // [V_SLOTS]
+    uint64_t* v_empty = bars + BAR_V_EMPTY;    // [V_SLOTS] (after P V)
+    uint64_t* p_full = bars + BAR_P_FULL;      // MMA -> mask
+    uint64_t* p_ready = bars + BAR_P_READY;    // mask -> MMA
+    uint64_t* ds_full = bars + BAR_DS_FULL;    // [2] MMA -> state
+    uint64_t* ds_empty = bars + BAR_DS_EMPTY;  // [2] state -> MMA
+    uint64_t* o_full = bars + BAR_O_FULL;      // [2] MMA -> output
+    uint64_t* o_empty = bars + BAR_O_EMPTY;    // [2] output -> MMA
+    uint64_t* s_full = bars + BAR_S_FULL;      // state -> MMA (S_hi/S_lo written)
+    uint64_t* s_empty = bars + BAR_S_EMPTY;    // MMA -> state (Q S product done)
+    uint64_t* drain = bars + BAR_DRAIN;        // MMA drain on exit
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + BAR_COUNT);
+    volatile int* abort = reinterpret_cast<volatile int*>(bars + BAR_COUNT + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -153,16 +179,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
+        for (int i = 0; i < QK_SLOTS; ++i) {
+            mbar_init(&qk_full[i], 1);
+            mbar_init(&qk_empty[i], 1);
+        }
+        for (int i = 0; i < V_SLOTS; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-            mbar_init(&p_full[i], 1);
-            mbar_init(&p_ready[i], 4);
             mbar_init(&ds_full[i], 1);
             mbar_init(&ds_empty[i], 4);
             mbar_init(&o_full[i], 1);
             mbar_init(&o_empty[i], 4);
         }
+        mbar_init(p_full, 1);
+        mbar_init(p_ready, 4);
         mbar_init(s_full, 4);
         mbar_init(s_empty, 1);
         mbar_init(drain, 1);
@@ -193,116 +225,161 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (idx >= p.n_items) break;
                 const Item it = decode_item(p, idx);
                 const int nc = (it.len + C - 1) / C;
-                bool stop = false;
-                for (int c = 0; c < nc; ++c, ++g) {
-                    const int st = g & 1, k = g >> 1;
-                    if (k > 0 && !mbar_wait(&empty[st], (k - 1) & 1, abort, p.status)) { stop = true; break; }
-                    mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
-                    uint8_t* sb = sm + st * STAGE_BYTES;
-                    int y, z;
+                auto coords = [&](int c, int& y, int& z) {
                     if (p.mode == 0) { y = c * C; z = it.c2; }
                     else { y = it.c1; z = it.t0 + c * C; }
-                    tma_load_3d(sb + OFF_Q, &map_q, &full[st], 0, y, z);
-                    tma_load_3d(sb + OFF_Q + PANEL, &map_q, &full[st], 64, y, z);
-                    tma_load_3d(sb + OFF_K, &map_k, &full[st], 0, y, z);
-                    tma_load_3d(sb + OFF_K + PANEL, &map_k, &full[st], 64, y, z);
-                    tma_load_3d(sb + OFF_V, &map_v, &full[st], DVS * it.vs, y, z);
+                };
+                auto prefetch = [&](int c) {
+                    int y, z;
+                    coords(c, y, z);
+                    tma_prefetch_3d(&map_q, 0, y, z);
+                    tma_prefetch_3d(&map_q, 64, y, z);
+                    tma_prefetch_3d(&map_k, 0, y, z);
+                    tma_prefetch_3d(&map_k, 64, y, z);
+                    tma_prefetch_3d(&map_v, DVS * it.vs, y, z);
+                };
+                for (int c = 0; c < PREFETCH && c < nc; ++c) prefetch(c);
+                bool stop = false;
+                for (int c = 0; c < nc; ++c, ++g) {
+                    if (c + PREFETCH < nc) prefetch(c + PREFETCH);
+                    int y, z;
+                    coords(c, y, z);
+                    const int a = g % QK_SLOTS, ka = g / QK_SLOTS;
+                    if (ka > 0 && !mbar_wait(&qk_empty[a], (ka - 1) & 1, abort, p.status)) { stop = true; break; }
+                    uint8_t* qk = sm + OFF_QK + a * QK_BYTES;
+                    mbar_arrive_expect_tx(&qk_full[a], QK_BYTES);
+                    tma_load_3d(qk, &map_q, &qk_full[a], 0, y, z);
+                    tma_load_3d(qk + PANEL, &map_q, &qk_full[a], 64, y, z);
+                    tma_load_3d(qk + 2 * PANEL, &map_k, &qk_full[a], 0, y, z);
+                    tma_load_3d(qk + 3 * PANEL, &map_k, &qk_full[a], 64, y, z);
+                    const int vc = g % V_SLOTS, kv = g / V_SLOTS;
+                    if (kv > 0 && !mbar_wait(&v_empty[vc], (kv - 1) & 1, abort, p.status)) { stop = true; break; }
+                    mbar_arrive_expect_tx(&v_full[vc], PANEL);
+                    tma_load_3d(sm + OFF_V + vc * PANEL, &map_v, &v_full[vc], DVS * it.vs, y, z);
                 }
                 if (stop) break;
             }
             // make sure no copy into shared memory is still in flight at exit
-            for (int x = (g >= 2 ? g - 2 : 0); x < g; ++x) drain_wait(&full[x & 1], (x >> 1) & 1);
+            for (int x = (g >= QK_SLOTS ? g - QK_SLOTS : 0); x < g; ++x)
+                drain_wait(&qk_full[x % QK_SLOTS], (x / QK_SLOTS) & 1);
+            for (int x = (g >= V_SLOTS ? g - V_SLOTS : 0); x < g; ++x)
+                drain_wait(&v_full[x % V_SLOTS], (x / V_SLOTS) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        const uint32_t id_p = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_ds = idesc_bf16(128, DVS, 1, 1);
-        const uint32_t id_pv = idesc_bf16(128, DVS, 0, 1);
-        const uint32_t id_qs = idesc_bf16(128, DVS, 0, 1);
-        const uint32_t s_hi = smem_u32(sm + OFF_SHI), s_lo = smem_u32(sm + OFF_SLO);
-        int g = 0;
-        bool stop = false;
-        for (int r = 0; !stop; ++r) {
-            const int idx = item_index(r, cta, G);
-            if (idx >= p.n_items) break;
-            const Item it = decode_item(p, idx);
-            const int nc = (it.len + C - 1) / C;
-            for (int c = 0; c < nc; ++c, ++g) {
-                const int st = g & 1, b = g & 1, k = g >> 1;
-                if (!warp_wait(&full[st], k & 1, abort, p.status)) { stop = true; break; }
-                uint8_t* sb = sm + st * STAGE_BYTES;
-                const int rows = it.len - c * C;
-                if (p.mode == 1 && rows < C) {
-                    // ragged tail inside a packed batch: rows past the end belong to
-                    // the next sequence; clear them in K and V before any product
-                    const int first = rows * 128;
-                    const int n16 = (PANEL - first) >> 4;
-                    for (int pnl = 0; pnl < 3; ++pnl) {
-                        uint8_t* base = sb + (pnl < 2 ? OFF_K + pnl * PANEL : OFF_V) + first;
-                        for (int e = lane; e < n16; e += 32)
-                            *reinterpret_cast<uint4*>(base + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+        // One thread issues every product; the other lanes of this warp only
+        // take part in TMEM allocation.  The tensor pipe is fed from this single
+        // thread, so each group of products is issued from fully unrolled code
+        // with its descriptors computed up front (a rolled loop only for the
+        // ragged last chunk of a packed sequence).  Completions of this thread's
+        // own tcgen05.commit need no fence; TMEM written or read by other warps is
+        // ordered by tcgen05.fence::after_thread_sync after the barrier.
+        if (lane == 0) {
+            constexpr uint32_t id_p = idesc_bf16(128, 128, 0, 0);   // Q K^T
+            constexpr uint32_t id_qs = idesc_bf16(128, 128, 0, 1);  // Q [S_hi | S_lo]
+            constexpr uint32_t id_ds = idesc_bf16(128, DVS, 1, 1);  // K^T V
+            constexpr uint32_t id_pv = idesc_bf16(128, DVS, 0, 1);  // P V (P from TMEM)
+            const uint64_t d_qk0 = sw128_desc(smem_u32(sm + OFF_QK), 16, 1024);
+            const uint64_t d_kt0 = sw128_desc(smem_u32(sm + OFF_QK + 2 * PANEL), PANEL, 1024);
+            const uint64_t d_v0 = sw128_desc(smem_u32(sm + OFF_V), PANEL, 1024);
+            const uint64_t d_s = sw128_desc(smem_u32(sm + OFF_SHI), PANEL, 1024);
+            const uint32_t tp = tbase + TM_P;
+            // K-step offsets (16-byte units): K-major tiles step 32 B inside a
+            // 64-column panel, MN-major tiles step 16 rows (2048 B)
+            auto kmaj = [](int kk) { return static_cast<uint64_t>(((kk >> 2) * PANEL + (kk & 3) * 32) >> 4); };
+            auto mnmaj = [](int kk) { return static_cast<uint64_t>((kk * 2048) >> 4); };
+            int g = 0;
+            bool stop = false;
+            for (int r = 0; !stop; ++r) {
+                const int idx = item_index(r, cta, G);
+                if (idx >= p.n_items) break;
+                const Item it = decode_item(p, idx);
+                const int nc = (it.len + C - 1) / C;
+                for (int c = 0; c < nc; ++c, ++g) {
+                    const int a = g % QK_SLOTS, ka = g / QK_SLOTS;
+                    const int vc = g % V_SLOTS, kv = g / V_SLOTS;
+                    const int b = g & 1, kb = g >> 1;
+                    const uint64_t d_q = d_qk0 + static_cast<uint64_t>((a * QK_BYTES) >> 4);
+                    const uint64_t d_k = d_q + static_cast<uint64_t>((2 * PANEL) >> 4);
+                    const uint64_t d_kt = d_kt0 + static_cast<uint64_t>((a * QK_BYTES) >> 4);
+                    const uint64_t d_v = d_v0 + static_cast<uint64_t>((vc * PANEL) >> 4);
+                    const uint32_t to = tbase + TM_O + 128u * b, tds = tbase + TM_DS + 64u * b;
+                    // a ragged tail inside a packed batch: rows past the end belong to
+                    // the next sequence.  Products over the token dim (K^T V, P V) stop
+                    // at the last 16-row step holding valid rows, whose invalid rows are
+                    // cleared; Q K^T columns past the end are removed by the causal mask.
+                    const int rows = it.len - c * C;
+                    const bool ragged = p.mode == 1 && rows < C;
+                    const int ksteps = ragged ? (rows + 15) >> 4 : C / 16;
+                    if (!mbar_wait(&qk_full[a], ka & 1, abort, p.status)) { stop = true; break; }
+                    if (ragged && (rows & 15)) {
+                        uint8_t* kb0 = sm + OFF_QK + a * QK_BYTES + 2 * PANEL;
+                        for (int pnl = 0; pnl < 2; ++pnl)
+                            for (int e = rows * 128; e < ksteps * 16 * 128; e += 16)
+                                *reinterpret_cast<uint4*>(kb0 + pnl * PANEL + e) = make_uint4(0u, 0u, 0u, 0u);
+                        fence_proxy_async_smem();
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                tc_fence_after();
-                const uint32_t qa = smem_u32(sb + OFF_Q), ka = smem_u32(sb + OFF_K), va = smem_u32(sb + OFF_V);
-                const uint32_t tp = tbase + TM_P + 128u * b, to = tbase + TM_O + 64u * b,
-                               tds = tbase + TM_DS + 64u * b;
-                if (lane == 0) {
                     // P = Q K^T   (A: Q K-major, B: K K-major)
+                    {
+                        uint64_t da[8], db[8];
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
-                        mma_ss(tp, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_p, kk > 0);
+                        for (int kk = 0; kk < 8; ++kk) { da[kk] = d_q + kmaj(kk); db[kk] = d_k + kmaj(kk); }
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) mma_ss(tp, da[kk], db[kk], id_p, kk > 0);
                     }
-                    mma_commit(&p_full[b]);
-                }
-                __syncwarp();
-                // dS = K^T V   (A: K MN-major over 2 panels, B: V MN-major)
-                if (k > 0 && !warp_wait(&ds_empty[b], (k - 1) & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                if (lane == 0) {
+                    mma_commit(p_full);
+                    // dS = K^T V   (A: K MN-major over 2 panels, B: V MN-major); issued
+                    // early so the state warps have the rest of this chunk and the
+                    // next chunk's P to fold it into S before the next Q S product
+                    if (!mbar_wait(&v_full[vc], kv & 1, abort, p.status)) { stop = true; break; }
+                    if (ragged && (rows & 15)) {
+                        uint8_t* vb = sm + OFF_V + vc * PANEL;
+                        for (int e = rows * 128; e < ksteps * 16 * 128; e += 16)
+                            *reinterpret_cast<uint4*>(vb + e) = make_uint4(0u, 0u, 0u, 0u);
+                        fence_proxy_async_smem();
+                    }
+                    if (kb > 0 && !mbar_wait(&ds_empty[b], (kb - 1) & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    if (!ragged) {
+                        uint64_t da[8], db[8];
 #pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        mma_ss(tds, sw128_desc(ka + kk * 2048, PANEL, 1024), sw128_desc(va + kk * 2048, PANEL, 1024),
-                               id_ds, kk > 0);
+                        for (int kk = 0; kk < 8; ++kk) { da[kk] = d_kt + mnmaj(kk); db[kk] = d_v + mnmaj(kk); }
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) mma_ss(tds, da[kk], db[kk], id_ds, kk > 0);
+                    } else {
+                        for (int kk = 0; kk < ksteps; ++kk) mma_ss(tds, d_kt + mnmaj(kk), d_v + mnmaj(kk), id_ds, kk > 0);
+                    }
                     mma_commit(&ds_full[b]);
-                }
-                __syncwarp();
-                // O = P V   (A: masked bf16 P in TMEM)
-                if (!warp_wait(&p_ready[b], k & 1, abort, p.status)) { stop = true; break; }
-                if (k > 0 && !warp_wait(&o_empty[b], (k - 1) & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                if (lane == 0) {
+                    // [O | O'] = Q [S_hi | S_lo]   (B: the two S panels, MN-major, N = 128)
+                    if (kb > 0 && !mbar_wait(&o_empty[b], (kb - 1) & 1, abort, p.status)) { stop = true; break; }
+                    if (!mbar_wait(s_full, g & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    {
+                        uint64_t da[8], db[8];
 #pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        mma_ts(to, tp + kk * 8, sw128_desc(va + kk * 2048, PANEL, 1024), id_pv, kk > 0);
-                }
-                __syncwarp();
-                // O += Q S_hi + Q S_lo   (B: S slices MN-major)
-                if (!warp_wait(s_full, g & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                if (lane == 0) {
+                        for (int kk = 0; kk < 8; ++kk) { da[kk] = d_q + kmaj(kk); db[kk] = d_s + mnmaj(kk); }
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
-                        mma_ss(to, sw128_desc(qa + off, 16, 1024), sw128_desc(s_hi + kk * 2048, PANEL, 1024), id_qs, 1);
+                        for (int kk = 0; kk < 8; ++kk) mma_ss(to, da[kk], db[kk], id_qs, kk > 0);
                     }
+                    mma_commit(s_empty);
+                    mma_commit(&qk_empty[a]);
+                    // O += P V   (A: masked bf16 P in TMEM, B: V MN-major)
+                    if (!mbar_wait(p_ready, g & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    if (!ragged) {
+                        uint64_t db[8];
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
-                        mma_ss(to, sw128_desc(qa + off, 16, 1024), sw128_desc(s_lo + kk * 2048, PANEL, 1024), id_qs, 1);
+                        for (int kk = 0; kk < 8; ++kk) db[kk] = d_v + mnmaj(kk);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) mma_ts(to, tp + kk * 8, db[kk], id_pv, 1);
+                    } else {
+                        for (int kk = 0; kk < ksteps; ++kk) mma_ts(to, tp + kk * 8, d_v + mnmaj(kk), id_pv, 1);
                     }
                     mma_commit(&o_full[b]);
-                    mma_commit(s_empty);
-                    mma_commit(&empty[st]);
+                    mma_commit(&v_empty[vc]);
                 }
-                __syncwarp();
             }
-        }
-        // every MMA issued by this thread must be finished before TMEM is freed
-        if (lane == 0) {
+            // every MMA issued by this thread must be finished before TMEM is freed
             mma_commit(drain);
             drain_wait(drain, 0);
         }
@@ -311,6 +388,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // ------------------------------------------------------ mask warps
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
+        const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_P;
         int g = 0;
         bool stop = false;
         for (int r = 0; !stop; ++r) {
@@ -319,34 +397,33 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             const Item it = decode_item(p, idx);
             const int nc = (it.len + C - 1) / C;
             for (int c = 0; c < nc; ++c, ++g) {
-                const int b = g & 1, k = g >> 1;
-                if (!warp_wait(&p_full[b], k & 1, abort, p.status)) { stop = true; break; }
+                if (!warp_wait(p_full, g & 1, abort, p.status)) { stop = true; break; }
                 tc_fence_after();
-                const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_P + 128u * b;
+                // columns s of 32-wide pieces 2h, 2h+1; pieces above this warp's rows are zero
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc) {
-                    uint32_t packed[16];
-                    if (pc > q4) {
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v0[32], v1[32];
+                    const int p0 = 2 * h, p1 = 2 * h + 1;
+                    if (p0 <= q4) tmem_ld32(ta + 32 * p0, v0);
+                    if (p1 <= q4) tmem_ld32(ta + 32 * p1, v1);
+                    if (p0 <= q4) tmem_wait_ld();
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                    } else {
-                        uint32_t v[32];
-                        tmem_ld32(ta + 32 * pc, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int s = 32 * pc + 2 * i;
-                            const float a0 = (s <= row) ? __uint_as_float(v[2 * i]) : 0.f;
-                            const float a1 = (s + 1 <= row) ? __uint_as_float(v[2 * i + 1]) : 0.f;
-                            packed[i] = pack_bf16x2(a0, a1);
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        const int s0 = 32 * p0 + 2 * i, s1 = 32 * p1 + 2 * i;
+                        pk[i] = (p0 <= q4) ? pack_bf16x2(s0 <= row ? __uint_as_float(v0[2 * i]) : 0.f,
+                                                         s0 + 1 <= row ? __uint_as_float(v0[2 * i + 1]) : 0.f)
+                                           : 0u;
+                        pk[16 + i] = (p1 <= q4) ? pack_bf16x2(s1 <= row ? __uint_as_float(v1[2 * i]) : 0.f,
+                                                              s1 + 1 <= row ? __uint_as_float(v1[2 * i + 1]) : 0.f)
+                                                : 0u;
                     }
-                    tmem_st16(ta + 16 * pc, packed);
+                    tmem_st32(ta + 32 * h, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_ready[b]);
+                if (lane == 0) mbar_arrive(p_ready);
             }
         }
     } else if (warp < 10) {
@@ -375,7 +452,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int j = 0; j < DVS; ++j) S[j] = 0.f;
             }
             for (int c = 0; c < nc; ++c, ++g) {
-                const int b = g & 1, k = g >> 1;
+                const int b = g & 1, kb = g >> 1;
                 // publish S_{c-1} as S_hi + S_lo (bf16, MN-major swizzled rows)
                 if (g > 0 && !warp_wait(s_empty, (g - 1) & 1, abort, p.status)) { stop = true; break; }
 #pragma unroll
@@ -396,20 +473,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_full);
                 // absorb dS_c
-                if (!warp_wait(&ds_full[b], k & 1, abort, p.status)) { stop = true; break; }
+                if (!warp_wait(&ds_full[b], kb & 1, abort, p.status)) { stop = true; break; }
                 tc_fence_after();
                 const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_DS + 64u * b;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + 32 * h2, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) S[32 * h2 + j] += __uint_as_float(v[j]);
-                }
+                uint32_t v0[32], v1[32];
+                tmem_ld32(ta, v0);
+                tmem_ld32(ta + 32, v1);
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ds_empty[b]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    S[j] += __uint_as_float(v0[j]);
+                    S[32 + j] += __uint_as_float(v1[j]);
+                }
             }
             if (stop) break;
             if (p.s_out) {
@@ -423,6 +501,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // ------------------------------------------------------ output warps
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
+        uint8_t* stg = sm + OFF_OST + q4 * 32 * 128;  // this warp's 32 staging rows
         int g = 0;
         bool stop = false;
         for (int r = 0; !stop; ++r) {
@@ -431,19 +510,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             const Item it = decode_item(p, idx);
             const int nc = (it.len + C - 1) / C;
             for (int c = 0; c < nc; ++c, ++g) {
-                const int b = g & 1, k = g >> 1;
-                if (!warp_wait(&o_full[b], k & 1, abort, p.status)) { stop = true; break; }
+                const int b = g & 1, kb = g >> 1;
+                if (!warp_wait(&o_full[b], kb & 1, abort, p.status)) { stop = true; break; }
                 tc_fence_after();
-                const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_O + 64u * b;
+                const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_O + 128u * b;
                 uint32_t hp[32];
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + 32 * h2, v);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(ta + 32 * h, v0);       // Q S_hi + P V
+                    tmem_ld32(ta + 64 + 32 * h, v1);  // Q S_lo
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        hp[16 * h2 + e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                        hp[16 * h + e] = pack_bf16x2(__uint_as_float(v0[2 * e]) + __uint_as_float(v1[2 * e]),
+                                                     __uint_as_float(v0[2 * e + 1]) + __uint_as_float(v1[2 * e + 1]));
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -453,8 +534,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     // this warp's rows all lie past the end of the sequence
                 } else if (p.mode == 0 || rows >= C) {
                     // each warp stages its 32 rows and stores them with one TMA copy
-                    uint8_t* stg = sm + OFF_OST + (g & 1) * PANEL + q4 * 32 * 128;
-                    if (lane == 0) bulk_wait_read<1>();
+                    if (lane == 0) bulk_wait_read<0>();
                     __syncwarp();
                     const uint32_t sa = smem_u32(stg) + static_cast<uint32_t>(lane) * 128u;
 #pragma unroll
@@ -469,6 +549,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         bulk_commit();
                     }
                 } else if (row < rows) {
+                    // ragged tail of a packed sequence: plain row stores
                     uint4* dst = reinterpret_cast<uint4*>(
                         p.o + ((long)(it.t0 + c * C + row) * p.H + it.c1) * p.dv + DVS * it.vs);
 #pragma unroll
