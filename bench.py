@@ -43,6 +43,15 @@ VARLEN = dict(n_seq=64, lo=1024, hi=32768, H=32, d=128, n_resume=32, prefix=4096
 PREFILL8K = dict(B=4, H=32, N=8192, d=128)
 METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 
+# DRAM traffic of one prefill launch, from one ncu capture (dram__bytes_read.sum
+# + dram__bytes_write.sum) of the kernel built from sources with this hash, on
+# the H=16, N=32768 case: 517.36 MB for 16*32768 token-heads.  Traffic grows
+# with the token-head count, so a launch is scaled by its token-heads.  When the
+# kernel sources change the figure no longer applies and is reported as null.
+TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
+TRAFFIC_HASH = "263cc8b75975a819"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = 517.36e6 / (16 * 32768)
+
 
 # ----------------------------------------------------------------- helpers
 def peaks():
@@ -159,6 +168,17 @@ def flops_issued(tokens_heads: float, d: int, C: int = 128, slice_w: int = 64) -
     return tokens_heads * n_vs * (2 * C * d + 2 * C * slice_w + 4 * d * slice_w + 2 * d * slice_w)
 
 
+def measured_traffic(token_heads: float):
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != TRAFFIC_HASH:
+        return None
+    return TRAFFIC_BYTES_PER_TOKEN_HEAD * token_heads
+
+
 def prefill_bytes(B, H, N, d) -> float:
     """Algorithmic HBM bytes: read Q, K, V, write O (bf16), write S (fp32)."""
     return 4.0 * B * H * N * d * 2 + B * H * d * d * 4
@@ -245,6 +265,7 @@ def run_headline(args, dist: Dist, pk, sampler: ClockSampler):
     del q, k, v, o, s
     torch.cuda.empty_cache()
     res = dict(value=value, ms_per_step=ms_step, launch_ms=launch_ms, achieved_gbs=achieved_gbs,
+               traffic=measured_traffic(th),
                bytes_launch=bytes_launch, tflops_rec=f_rec, tflops_issued=f_iss, clocks=clocks, e2e=e2e,
                launches=args.steps)
     return res, sample
@@ -457,7 +478,7 @@ def main():
                         l2="inputs larger than L2, no flush" if 3 * args.heads * args.seq * d * 2 > 126e6
                         else "inputs fit in L2 (profiling case)"),
             roofline=dict(bound="hbm", achieved=head["achieved_gbs"], peak=pk["hbm"], unit="GB/s",
-                          frac=head["achieved_gbs"] / pk["hbm"], traffic=None, peak_source=peak_note,
+                          frac=head["achieved_gbs"] / pk["hbm"], traffic=head["traffic"], peak_source=peak_note,
                           algorithmic_bytes_per_launch=head["bytes_launch"], launch_ms=head["launch_ms"]),
             tensor=dict(tflops_rec=head["tflops_rec"], tflops_issued=head["tflops_issued"],
                         frac_rec=head["tflops_rec"] / pk["bf16"], frac_issued=head["tflops_issued"] / pk["bf16"],
