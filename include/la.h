@@ -132,6 +132,40 @@ LA_API la_status la_decode_step(const void* q, const void* k, const void* v, voi
  */
 LA_API la_status la_device_status(int* out, int clear);
 
+/*
+ * Ragged prefill for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for library users.
+ * la_prefill_varlen needs a caller-provided device workspace (it sorts the
+ * sequences by length on the GPU).  Some callers cannot obtain one at call
+ * time: code embedded in a host framework that owns all device memory and
+ * offers no allocator at that point, or latency-critical serving loops where
+ * cudaMalloc/cudaFree (which may synchronize the device) are not allowed.
+ * This entry point takes the same arguments minus the workspace and uses a
+ * scratch array built into the library instead: a file-scope device array of
+ * LA_NOALLOC_MAX_SEQS 32-bit entries that every GPU loading the library holds
+ * until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ *  - n_seq > LA_NOALLOC_MAX_SEQS returns LA_ERR_INVALID_ARG (use
+ *    la_prefill_varlen with a workspace for larger batches).
+ *  - All calls on a device share the one scratch array and it keeps the last
+ *    call's contents (every call rewrites the part it reads).  Calls whose
+ *    work overlaps on the GPU (different streams, or different host threads,
+ *    without ordering between them) race on it: order them on one stream.
+ *  - The first call on each device performs a one-time set-up on the host
+ *    (it looks up the device address of the scratch array for the current
+ *    device); make that first call before any stream capture.
+ * Everything else (arguments, layouts, results, errors) is as for
+ * la_prefill_varlen.
+ */
+#define LA_NOALLOC_MAX_SEQS 4096
+LA_API la_status la_prefill_varlen_noalloc(const void* q, const void* k, const void* v, void* o,
+                                           const int32_t* cu_seqlens, int n_seq, int T,
+                                           const float* state_pool, int n_pool, const int32_t* init_idx,
+                                           float* s_out, int H, int dk, int dv, la_dtype dt, int chunk,
+                                           la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

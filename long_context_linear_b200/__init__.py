@@ -19,8 +19,8 @@ import torch
 from . import _abi
 from ._abi import LAError, lib
 
-__all__ = ["prefill", "prefill_varlen", "decode_step", "device_status", "LAError", "lib",
-           "prefill_workspace_size", "prefill_varlen_workspace_size"]
+__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "decode_step", "device_status", "LAError",
+           "lib", "prefill_workspace_size", "prefill_varlen_workspace_size"]
 
 _DT = {torch.bfloat16: _abi.LA_BF16, torch.float32: _abi.LA_FP32}
 
@@ -141,6 +141,35 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
                                          chunk, _ptr(workspace), ws_bytes, _stream(q.device)),
                    "la_prefill_varlen")
     return out, s_out
+
+
+def prefill_varlen_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                           state_pool: Optional[torch.Tensor] = None, init_idx: Optional[torch.Tensor] = None, *,
+                           out: torch.Tensor, s_out: Optional[torch.Tensor] = None, chunk: int = 0) -> None:
+    """prefill_varlen for callers that cannot allocate device memory.
+
+    The caller passes every output buffer; the library uses its built-in
+    scratch (at most ``_abi.NOALLOC_MAX_SEQS`` sequences per call) instead of a
+    workspace.  Calls share that scratch: order them on one stream.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, n, q.dtype, q.device)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, q.device)
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n_seq = cu_seqlens.numel() - 1
+    n_pool = 0 if state_pool is None else state_pool.shape[0]
+    if state_pool is not None:
+        _need(state_pool, "state_pool", torch.float32, q.device)
+    if init_idx is not None:
+        _need(init_idx, "init_idx", torch.int32, q.device)
+    if s_out is not None:
+        _need(s_out, "s_out", torch.float32, q.device)
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_prefill_varlen_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq, T,
+                                                 _ptr(state_pool), n_pool, _ptr(init_idx), _ptr(s_out), H, dk, dv,
+                                                 _dtype_code(q), chunk, _stream(q.device)),
+                   "la_prefill_varlen_noalloc")
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,

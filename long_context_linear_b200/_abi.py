@@ -34,7 +34,10 @@ SIGNATURES = {
                                _vp, _sz, _vp]),
     "la_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
+    "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
+
+NOALLOC_MAX_SEQS = 4096  # LA_NOALLOC_MAX_SEQS in include/la.h
 
 
 class LAError(RuntimeError):

@@ -29,6 +29,12 @@ namespace lcl {
 // Device status word: 0, or LA_ERR_TIMEOUT after a bounded wait ran out.
 __device__ int g_status_word = 0;
 
+// Scratch used by la_prefill_varlen_noalloc in place of a caller workspace:
+// the longest-first sequence order of one packed batch.  One copy per device,
+// alive for the whole process; host code must look up its device address
+// (the array's name is only a host-side stand-in).
+static __device__ __align__(256) int g_noalloc_order[LA_NOALLOC_MAX_SEQS];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -385,6 +391,50 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o, f
         else dec::decode_step_kernel<T, 64><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
     }
     return after_launch("decode_step launch");
+}
+
+namespace lcl {
+namespace {
+int* g_noalloc_ptr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// One-time per-device set-up: the device address of g_noalloc_order for the
+// current device.
+la_status noalloc_scratch(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_order)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        g_noalloc_ptr[dev] = static_cast<int*>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return LA_OK;
+}
+}  // namespace
+}  // namespace lcl
+
+extern "C" la_status la_prefill_varlen_noalloc(const void* q, const void* k, const void* v, void* o,
+                                               const int32_t* cu_seqlens, int n_seq, int T,
+                                               const float* state_pool, int n_pool, const int32_t* init_idx,
+                                               float* s_out, int H, int dk, int dv, la_dtype dt, int chunk,
+                                               la_stream_t stream) {
+    g_last_error[0] = 0;
+    if (n_seq > LA_NOALLOC_MAX_SEQS)
+        return fail(LA_ERR_INVALID_ARG,
+                    "n_seq = %d exceeds the %d sequences the built-in scratch holds; "
+                    "use la_prefill_varlen with a workspace",
+                    n_seq, LA_NOALLOC_MAX_SEQS);
+    if (n_seq < 0) return fail(LA_ERR_INVALID_ARG, "negative size n_seq=%d", n_seq);
+    int* scratch = nullptr;
+    la_status s = noalloc_scratch(&scratch);
+    if (s != LA_OK) return s;
+    return la_prefill_varlen(q, k, v, o, cu_seqlens, n_seq, T, state_pool, n_pool, init_idx, s_out, H, dk, dv, dt,
+                             chunk, scratch, sizeof(int) * LA_NOALLOC_MAX_SEQS, stream);
 }
 
 la_status la_device_status(int* out, int clear) {
