@@ -66,35 +66,36 @@ def peaks():
 
 
 class Dist:
+    """One process per GPU (torchrun env vars); timing reductions over ranks."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cuda"
 
     def init(self, backend="nccl"):
         if self.world > 1:
             import torch.distributed as dist
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
             self.pg = dist
+            self.device = "cuda" if backend == "nccl" else "cpu"
 
     def barrier(self):
         if self.pg:
             self.pg.barrier()
 
-    def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+    def _reduce(self, x: float, op) -> float:
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=op)
         return float(t.item())
 
+    def max(self, x: float) -> float:
+        return x if not self.pg else self._reduce(x, self.pg.ReduceOp.MAX)
+
     def sum(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
-        return float(t.item())
+        return x if not self.pg else self._reduce(x, self.pg.ReduceOp.SUM)
 
     def close(self):
         if self.pg:
@@ -153,6 +154,12 @@ class ClockSampler:
         load = [s for s in sm if mx and s >= 0.5 * max(mx)] or sm
         return dict(sm_mhz=statistics.median(load) if load else None, sm_max_mhz=max(mx) if mx else None,
                     reasons=reasons, samples=len(rows), power_w_max=max(power) if power else None)
+
+
+def weak_scaling_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own units_per_rank in the
+    timed region, which lasts as long as the slowest rank (max_ms)."""
+    return units_per_rank * world / (max_ms / 1e3)
 
 
 def flops_rec(tokens_heads: float, d: int) -> float:
@@ -228,7 +235,7 @@ def run_headline(args, dist: Dist, pk, sampler: ClockSampler):
     launch_ms = dist.max(statistics.fmean(per_launch))
     ms_step = total_ms / args.steps
     tokens = B * N * dist.world
-    value = tokens / (ms_step / 1e3)
+    value = weak_scaling_rate(B * N, dist.world, ms_step)
     if (H, N) != (HEADLINE["H"], HEADLINE["N"]):
         print(f"note: headline workload overridden to H={H} N={N}", file=sys.stderr)
     th = B * H * N

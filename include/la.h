@@ -133,6 +133,15 @@ LA_API la_status la_decode_step(const void* q, const void* k, const void* v, voi
 LA_API la_status la_device_status(int* out, int clear);
 
 /*
+ * Self-test of device-side failure detection: launches one small kernel whose
+ * bounded wait can never be satisfied; after `timeout_us` microseconds
+ * (1 ..= 1,000,000) it gives up and records LA_ERR_TIMEOUT in the device status
+ * word (read it with la_device_status).  The context stays usable.  This is
+ * the same bounded-wait path every compute kernel takes when a wait runs out.
+ */
+LA_API la_status la_selftest_wait_timeout(int timeout_us, la_stream_t stream);
+
+/*
  * Ragged prefill for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this call; it exists for library users.

@@ -34,6 +34,7 @@ SIGNATURES = {
                                _vp, _sz, _vp]),
     "la_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
+    "la_selftest_wait_timeout": (_i, [_i, _vp]),
     "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
 

@@ -23,6 +23,7 @@
 #include "prefill_simt.cuh"
 #include "decode.cuh"
 #include "varlen_order.cuh"
+#include "selftest.cuh"
 
 namespace lcl {
 
@@ -435,6 +436,18 @@ extern "C" la_status la_prefill_varlen_noalloc(const void* q, const void* k, con
     if (s != LA_OK) return s;
     return la_prefill_varlen(q, k, v, o, cu_seqlens, n_seq, T, state_pool, n_pool, init_idx, s_out, H, dk, dv, dt,
                              chunk, scratch, sizeof(int) * LA_NOALLOC_MAX_SEQS, stream);
+}
+
+la_status la_selftest_wait_timeout(int timeout_us, la_stream_t stream) {
+    g_last_error[0] = 0;
+    if (timeout_us < 1 || timeout_us > 1000000)
+        return fail(LA_ERR_INVALID_ARG, "timeout_us = %d outside [1, 1000000]", timeout_us);
+    DeviceInfo* di;
+    la_status s = device_info(&di);
+    if (s != LA_OK) return s;
+    selftest::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<unsigned long long>(timeout_us) * 1000ull, di->status);
+    return after_launch("selftest launch");
 }
 
 la_status la_device_status(int* out, int clear) {

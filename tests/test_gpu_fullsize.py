@@ -1,0 +1,119 @@
+"""Parity at the full benchmark sizes, in the launch configuration bench.py times.
+
+Each test runs the whole batch through the C ABI exactly as the benchmark does
+(same shapes, same calls) and compares seeded samples of (batch, head) units
+against the fp64 oracle, which computes those units one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.parity import assert_out, assert_state, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def la():
+    import long_context_linear_b200 as la
+    return la
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def test_prefill_b4_h32_n8192(la, oracle_mod):
+    B, H, N, d = 4, 32, 8192, 128
+    dev = torch.device("cuda")
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=61, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    la.prefill(q, k, v, None, out=o, s_out=s)
+    assert la.device_status() == 0
+    units = synth.choose(B * H, 16, seed=1)
+    qf, kf, vf, of, sf = (x.view(B * H, *x.shape[2:]) for x in (q, k, v, o, s))
+    idx = torch.tensor(units, device=dev)
+    ro, rs = oracle_mod.recurrent(qf[idx].cpu(), kf[idx].cpu(), vf[idx].cpu())
+    assert_out(of[idx].cpu(), ro, torch.bfloat16, 1)
+    assert_state(sf[idx].cpu(), rs, 1)
+    del q, k, v, o, s
+    _free()
+
+
+def test_long_prefill_h64_n131072(la, oracle_mod):
+    B, H, N, d = 1, 64, 131072, 128
+    dev = torch.device("cuda")
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=3, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    la.prefill(q, k, v, None, out=o, s_out=s)
+    assert la.device_status() == 0
+    heads = synth.choose(H, 4, seed=2)
+    idx = torch.tensor(heads, device=dev)
+    ro, rs = oracle_mod.recurrent(q[0, idx].cpu(), k[0, idx].cpu(), v[0, idx].cpu())
+    assert_out(o[0, idx].cpu(), ro, torch.bfloat16, 1)
+    assert_state(s[0, idx].cpu(), rs, 1)
+    del q, k, v, o, s
+    _free()
+
+
+def test_decode_b256_h64_1024_steps(la, oracle_mod):
+    B, H, d, steps = 256, 64, 128, 1024
+    dev = torch.device("cuda")
+    U = B * H
+    L_seq = synth.lengths(B, 1024, 65536, seed=41)
+    L = [L_seq[u // H] for u in range(U)]
+    S = torch.empty(U, d, d, dtype=torch.float32, device=dev)
+    for u0 in range(0, U, 2048):
+        S[u0:u0 + 2048] = synth.outer_product_state(min(2048, U - u0), d, d, L[u0:u0 + 2048], seed=7 + u0,
+                                                    device=dev)
+    S = S.view(B, H, d, d)
+    units = synth.choose(U, 64, seed=3)
+    idx = torch.tensor(units, device=dev)
+    S_ref = S.view(U, d, d)[idx].double().cpu().numpy()
+    qs, ks, vs = synth.qkv((steps, B, H, d), d, "bf16", seed=43, device=dev)
+    o = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    check = {0, 1, 511, 1023}
+    for t in range(steps):
+        la.decode_step(qs[t], ks[t], vs[t], S, out=o)
+        qt, kt, vt = (x[t].view(U, d)[idx].cpu() for x in (qs, ks, vs))
+        ro, S_ref = oracle_mod.decode(qt, kt, vt, S_ref)
+        if t in check:
+            assert_out(o.view(U, d)[idx].cpu(), ro, torch.bfloat16, 1)
+    assert la.device_status() == 0
+    assert_state(S.view(U, d, d)[idx].cpu(), S_ref, 1, tol=1e-5)
+    del qs, ks, vs, S, o
+    _free()
+
+
+def test_varlen_64_sequences_with_resume(la, oracle_mod):
+    n_seq, H, d = 64, 32, 128
+    dev = torch.device("cuda")
+    lens = synth.lengths(n_seq, 1024, 32768, seed=51)
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=53, device=dev)
+    resumed = synth.choose(n_seq, 32, seed=55)
+    pool = synth.outer_product_state(32 * H, d, d, [4096] * (32 * H), seed=57, device=dev).view(32, H, d, d)
+    init = torch.full((n_seq,), -1, dtype=torch.int32)
+    for j, n in enumerate(resumed):
+        init[n] = j
+    o, s = la.prefill_varlen(q, k, v, cu.to(dev), pool, init.to(dev))
+    assert la.device_status() == 0
+    seqs = synth.choose(n_seq, 4, seed=4)
+    heads = synth.choose(H, 2, seed=5)
+    for n in seqs:
+        a, b = int(cu[n]), int(cu[n + 1])
+        hs = torch.tensor(heads, device=dev)
+        qn = q[a:b][:, hs].transpose(0, 1).cpu()
+        kn = k[a:b][:, hs].transpose(0, 1).cpu()
+        vn = v[a:b][:, hs].transpose(0, 1).cpu()
+        s0 = pool[int(init[n])][hs].cpu() if init[n] >= 0 else None
+        ro, rs = oracle_mod.recurrent(qn, kn, vn, s0)
+        assert_out(o[a:b][:, hs].transpose(0, 1).cpu(), ro, torch.bfloat16, 1)
+        assert_state(s[n][hs].cpu(), rs, 1)
+    del q, k, v, o, s, pool
+    _free()
