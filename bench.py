@@ -170,9 +170,9 @@ def flops_rec(tokens_heads: float, d: int) -> float:
 
 def flops_issued(tokens_heads: float, d: int, C: int = 128, slice_w: int = 64) -> float:
     """FLOPs the tensor cores execute: per 64-wide value slice, Q K^T (2 C d),
-    P V (2 C w), Q S_hi + Q S_lo (4 d w) and K^T V (2 d w) per token."""
+    Q S (2 d w), P V (2 C w) and K^T V (2 d w) per token."""
     n_vs = d // slice_w
-    return tokens_heads * n_vs * (2 * C * d + 2 * C * slice_w + 4 * d * slice_w + 2 * d * slice_w)
+    return tokens_heads * n_vs * (2 * C * d + 2 * d * slice_w + 2 * C * slice_w + 2 * d * slice_w)
 
 
 def measured_traffic(token_heads: float):

@@ -247,8 +247,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
 
     tc::Params p{};
     p.mode = 0;
-    p.n_vs = dv / tc::DVS;
-    p.n_items = (int)(U * p.n_vs);
+    p.n_items = (int)(U * tc::NVS);
     p.H = H;
     p.N = N;
     p.dv = dv;
@@ -342,8 +341,7 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
 
     tc::Params p{};
     p.mode = 1;
-    p.n_vs = dv / tc::DVS;
-    p.n_items = (int)((long)n_seq * H * p.n_vs);
+    p.n_items = (int)((long)n_seq * H * tc::NVS);
     p.H = H;
     p.dv = dv;
     p.cu_seqlens = cu_seqlens;

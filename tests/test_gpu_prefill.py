@@ -59,9 +59,10 @@ def test_tc_chunk_argument(la, oracle_mod, chunk):
 
 def test_tc_integer_inputs_bit_exact(la, oracle_mod):
     """Inputs in {-1,0,1}: every product and partial sum on the tensor-core
-    path is an exactly representable integer (|S| < 2^16 splits exactly into
-    bf16 hi + lo; fp32 sums stay below 2^24), so O must equal the bf16
-    rounding of the exact result and S must equal it bit for bit."""
+    path is an exactly representable integer (the running state stays well
+    inside |S| <= 256, where bf16(S) is exact; fp32 sums stay below 2^24), so
+    O must equal the bf16 rounding of the exact result and S must equal it bit
+    for bit."""
     B, H, N, d = 1, 2, 1000, 128
     q = synth.integer_valued((B, H, N, d), seed=1, dtype=torch.bfloat16)
     k = synth.integer_valued((B, H, N, d), seed=2, dtype=torch.bfloat16)
