@@ -468,15 +468,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // ------------------------------------------------------ state warps
         const int q4 = warp & 3;
         const int i = q4 * 32 + lane;  // key-dim row of S owned by this thread
-        const bool odd = lane & 1;
         const uint32_t ta0 = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_DS;
-        // S^T row j (value column j) sits at row C + j of each K panel, dk
-        // columns (i & ~1, i | 1) forming one 32-bit word.  The even lane of a
-        // pair writes that word for column j0 and the odd lane for j0 + 4, so
-        // one store instruction covers two rows in disjoint banks.
-        const uint32_t sel = odd ? 0x3276u : 0x5410u;
-        const uint32_t chunk_l = static_cast<uint32_t>((i & 63) >> 3) ^ (odd ? 4u : 0u);
-        const uint32_t row_l = static_cast<uint32_t>((i >> 6) * KPANEL + (C + (odd ? 4 : 0)) * 128 + (i & 6) * 2);
+        // S^T row j (value column j) sits at row C + j of each K panel; this
+        // thread writes the bf16 of S[i][j] at dk column i of every row.  A
+        // warp's 32 two-byte stores of one row fill 4 distinct 16-byte chunks.
+        const uint32_t colchunk = static_cast<uint32_t>((i & 63) >> 3);
+        const uint32_t col_off = static_cast<uint32_t>((i >> 6) * KPANEL + C * 128 + (i & 7) * 2);
         int g = 0;
         bool stop = false;
         for (int r = 0; !stop; ++r) {
@@ -499,17 +496,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 // publish bf16(S_{c-1})^T next to K_c, once the slot's previous product is done
                 const int ks = g % K_SLOTS;
                 if (g >= K_SLOTS && !warp_wait(&k_empty[ks], ((g / K_SLOTS) - 1) & 1, abort, p.status)) { stop = true; break; }
-                const uint32_t base = smem_u32(sm + OFF_K + ks * TILE_K) + row_l;
-                uint32_t addr[4];
+                uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
+                __nv_bfloat16* rowp[8];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) addr[m] = base + ((chunk_l ^ static_cast<uint32_t>(m)) << 4);
+                for (int m = 0; m < 8; ++m)
+                    rowp[m] = reinterpret_cast<__nv_bfloat16*>(base + ((colchunk ^ static_cast<uint32_t>(m)) << 4));
 #pragma unroll
-                for (int t = 0; t < DVS / 2; ++t) {
-                    const int j0 = (t >> 2) * 8 + (t & 3);
-                    const uint32_t w = pack_bf16x2(S[j0], S[j0 + 4]);
-                    const uint32_t w2 = __shfl_xor_sync(0xffffffffu, w, 1);
-                    st_shared_b32(addr[t & 3] + j0 * 128u, __byte_perm(w, w2, sel));
-                }
+                for (int j = 0; j < DVS; ++j) rowp[j & 7][j * 64] = __float2bfloat16_rn(S[j]);
                 fence_proxy_async_smem();
                 // the [P|O] product of this chunk also needs Q_c, K_c and the O
                 // buffer it writes (last used by chunk c - 2) drained
