@@ -181,6 +181,14 @@ __device__ __forceinline__ uint64_t mnmaj_desc(uint32_t base, int kk, uint32_t l
     return sw128_desc(base + static_cast<uint32_t>(kk) * 2048u, lbo, 1024);
 }
 
+// The same descriptors as K-step offsets (16-byte units) from the K-step-0
+// descriptor, for unrolled issue loops: the tcgen05.mma operands then need no
+// per-instruction address arithmetic in the issuing thread.
+__device__ __forceinline__ constexpr uint64_t kmaj_step(int kk, uint32_t panel) {
+    return static_cast<uint64_t>((static_cast<uint32_t>(kk >> 2) * panel + static_cast<uint32_t>(kk & 3) * 32u) >> 4);
+}
+__device__ __forceinline__ constexpr uint64_t mnmaj_step(int kk) { return static_cast<uint64_t>(kk) * (2048u >> 4); }
+
 // The code below is kept compact on purpose: all warps of all SMs run their
 // roles' loops at once, so the kernel's instruction footprint (not only its
 // instruction count) decides how often warps stall on instruction fetch.
@@ -352,10 +360,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         if (!mbar_wait(&s_full[ks], (k / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                         tc_fence_after();
                         const uint32_t tpo = tbase + TM_PO_STRIDE * b;
-                        const uint32_t qa = sq + qs * TILE_Q, ka = sk + ks * TILE_K;
-#pragma unroll 1
+                        const uint64_t da = kmaj_desc(sq + qs * TILE_Q, 0, PANEL);
+                        const uint64_t db = kmaj_desc(sk + ks * TILE_K, 0, KPANEL);
+#pragma unroll
                         for (int kk = 0; kk < DK / 16; ++kk)
-                            mma_ss(tpo, kmaj_desc(qa, kk, PANEL), kmaj_desc(ka, kk, KPANEL), id_f, kk > 0);
+                            mma_ss(tpo, da + kmaj_step(kk, PANEL), db + kmaj_step(kk, KPANEL), id_f, kk > 0);
                         mma_commit(&p_full[b]);
                         mma_commit(&q_empty[qs]);
                         mma_commit(&k_empty[ks]);
@@ -371,10 +380,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     if (ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
                     tc_fence_after();
                     const uint32_t tpo = tbase + TM_PO_STRIDE * b;
-                    const uint32_t va = sv + vc * PANEL;
+                    const uint64_t dv = mnmaj_desc(sv + vc * PANEL, 0, PANEL);
+                    if (ksteps == C / 16) {
+#pragma unroll
+                        for (int kk = 0; kk < C / 16; ++kk) mma_ts(tpo + TM_O_OFF, tpo + kk * 8, dv + mnmaj_step(kk), id_pv, 1);
+                    } else {
 #pragma unroll 1
-                    for (int kk = 0; kk < ksteps; ++kk)
-                        mma_ts(tpo + TM_O_OFF, tpo + kk * 8, mnmaj_desc(va, kk, PANEL), id_pv, 1);
+                        for (int kk = 0; kk < ksteps; ++kk) mma_ts(tpo + TM_O_OFF, tpo + kk * 8, dv + mnmaj_step(kk), id_pv, 1);
+                    }
                     mma_commit(&o_full[b]);
                     mma_commit(&v_empty[vc]);
                 }
@@ -408,10 +421,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     if (g >= 2 && !mbar_wait(&ds_empty[b], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
                     const uint32_t tds = tbase + TM_DS + TM_PO_STRIDE * b;
-                    const uint32_t ka = sk + ks * TILE_K, va = sv + vc * PANEL;
+                    const uint64_t dk = mnmaj_desc(sk + ks * TILE_K, 0, KPANEL), dv = mnmaj_desc(sv + vc * PANEL, 0, PANEL);
+                    if (ksteps == C / 16) {
+#pragma unroll
+                        for (int kk = 0; kk < C / 16; ++kk) mma_ss(tds, dk + mnmaj_step(kk), dv + mnmaj_step(kk), id_ds, kk > 0);
+                    } else {
 #pragma unroll 1
-                    for (int kk = 0; kk < ksteps; ++kk)
-                        mma_ss(tds, mnmaj_desc(ka, kk, KPANEL), mnmaj_desc(va, kk, PANEL), id_ds, kk > 0);
+                        for (int kk = 0; kk < ksteps; ++kk) mma_ss(tds, dk + mnmaj_step(kk), dv + mnmaj_step(kk), id_ds, kk > 0);
+                    }
                     mma_commit(&ds_full[b]);
                     mma_commit(&k_empty[ks]);
                     mma_commit(&v_empty[vc]);
