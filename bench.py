@@ -45,12 +45,12 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 
 # DRAM traffic of one prefill launch, from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum) of the kernel built from sources with this hash, on
-# the H=16, N=32768 case: 517.36 MB for 16*32768 token-heads.  Traffic grows
+# the H=16, N=32768 case: 517.80 MB for 16*32768 token-heads.  Traffic grows
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "263cc8b75975a819"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = 517.36e6 / (16 * 32768)
+TRAFFIC_HASH = "2bf09d47bbe89457"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.73e6 + 115.07e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
