@@ -41,6 +41,7 @@ HEADLINE = dict(B=1, H=64, N=131072, d=128)
 DECODE = dict(B=256, H=64, d=128, steps=1024, L_lo=1024, L_hi=65536)
 VARLEN = dict(n_seq=64, lo=1024, hi=32768, H=32, d=128, n_resume=32, prefix=4096)
 PREFILL8K = dict(B=4, H=32, N=8192, d=128)
+FEWHEADS = dict(B=1, H=8, N=131072, d=128)  # under-filled grid: the segment split applies
 METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 
 # DRAM traffic of one prefill launch, from one ncu capture (dram__bytes_read.sum
@@ -378,6 +379,47 @@ def run_prefill8k(args, dist: Dist, pk):
                 l2="inputs (1 GiB) larger than L2")
 
 
+def run_few_heads(args, dist: Dist, pk):
+    """Long prefill with too few (batch, head) units to fill the GPU, once with
+    the library's segment split and once with it turned off."""
+    import long_context_linear_b200 as la
+    import synth
+    c = FEWHEADS
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=71 + dist.rank, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    ws_bytes = la.prefill_workspace_size(B, H, N, d, torch.bfloat16)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = max(10, min(args.steps, 50))
+    res = dict(workload="prefill B=1 H=8 N=131072 d=128 bf16 (16 value-slice items on 148 SMs)",
+               workspace_bytes=ws_bytes, steps=n)
+    byts = prefill_bytes(B, H, N, d)
+    prev = os.environ.get("LA_PREFILL_SEGMENTS")
+    try:
+        for key, env in (("split", None), ("unsplit", "1")):
+            if env is None:
+                os.environ.pop("LA_PREFILL_SEGMENTS", None)
+            else:
+                os.environ["LA_PREFILL_SEGMENTS"] = env
+            total_ms, _ = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, workspace=ws), n,
+                                         max(3, args.warmup), dist, stream)
+            ms_step = dist.max(total_ms) / n
+            gbs = byts / (ms_step / 1e3) / 1e9
+            res[key] = dict(ms_per_step=ms_step, tokens_per_s=B * N * dist.world / (ms_step / 1e3), hbm_gbs=gbs,
+                            frac=gbs / pk["hbm"])
+    finally:
+        if prev is None:
+            os.environ.pop("LA_PREFILL_SEGMENTS", None)
+        else:
+            os.environ["LA_PREFILL_SEGMENTS"] = prev
+    del q, k, v, o, s, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------- oracle arm
 def oracle_sample_plan(budget_s: float):
     """Heads x tokens of the headline workload the oracle processes in about
@@ -468,6 +510,7 @@ def main():
         extras["decode"] = run_decode(args, dist, pk)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
+        extras["few_heads"] = run_few_heads(args, dist, pk)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_line()

@@ -85,7 +85,16 @@ LA_API int la_version(void);
  *          FFMA path: 32 or 64 (default 64).  C does not change the result
  *          beyond rounding.
  *   workspace/ws_bytes: scratch of at least la_prefill_workspace_size(...)
- *          bytes (may be NULL when that size is 0).
+ *          bytes, 16-byte aligned (may be NULL when that size is 0).  The size
+ *          is non-zero when B*H units are too few to fill the GPU and N is
+ *          long: the tensor-core path then cuts each sequence into segments of
+ *          whole chunks (a segment split of the tiled form on page "MiniMax:
+ *          «Почему M2 в итоге стала моделью с полным вниманием?»", section 1,
+ *          glossary entry "Lightning Attention": the K^T V sums of the
+ *          segments give every segment its starting state).  The workspace
+ *          holds those fp32 states; with a NULL or smaller workspace the call
+ *          runs unsplit and still returns the same result.  The environment
+ *          variable LA_PREFILL_SEGMENTS=<n> forces n segments (1 = unsplit).
  * N = 0 writes s_out = s0 (or zero).  Returns LA_OK once enqueued.
  */
 LA_API size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt);

@@ -24,6 +24,7 @@
 #include "decode.cuh"
 #include "varlen_order.cuh"
 #include "selftest.cuh"
+#include "seg_prefix.cuh"
 
 namespace lcl {
 
@@ -213,15 +214,51 @@ const char* la_last_error(void) { return g_last_error; }
 
 int la_version(void) { return 100; }
 
+namespace {
+
+// Segment split of the dense tensor-core prefill: when the (unit, value slice)
+// items fill less than half of the SMs, each unit's sequence is cut into
+// segments of whole chunks (at least kMinSegChunks) so that about one item per
+// SM remains.  LA_PREFILL_SEGMENTS=<n> overrides the count (1 = no split).
+constexpr int kMinSegChunks = 8;
+
+int plan_segments(long U, int N, int sms, int* seg_len) {
+    const int nch = (N + tc::C - 1) / tc::C;
+    *seg_len = nch * tc::C;
+    if (N <= 0) return 1;
+    int P;
+    if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
+        P = atoi(e);
+    } else {
+        const long items = U * tc::NVS;
+        P = items * 2 > sms ? 1 : (int)(sms / items);
+        P = std::min(P, nch / kMinSegChunks);
+    }
+    P = std::max(1, std::min(P, nch));
+    const int cps = (nch + P - 1) / P;  // chunks per segment
+    *seg_len = cps * tc::C;
+    return (nch + cps - 1) / cps;
+}
+
+size_t segment_workspace_bytes(long U, int P, int dk, int dv) {
+    if (P <= 1) return 0;
+    return (size_t)U * (size_t)(2 * P - 1) * (size_t)dk * (size_t)dv * sizeof(float);
+}
+
+}  // namespace
+
 size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt) {
-    (void)B; (void)H; (void)N; (void)dk; (void)dv; (void)dt;
-    return 0;
+    if (B <= 0 || H <= 0 || N <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return 0;
+    DeviceInfo* di;
+    if (device_info(&di) != LA_OK) return 0;
+    int seg_len;
+    const long U = (long)B * H;
+    return segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), dk, dv);
 }
 
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
                      int H, int N, int dk, int dv, la_dtype dt, int chunk, void* workspace, size_t ws_bytes,
                      la_stream_t stream) {
-    (void)workspace; (void)ws_bytes;
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
@@ -255,7 +292,17 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     p.s_out = s_out;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.status = di->status;
+    p.n_seg = 1;
     if (N == 0 && !s_out) return LA_OK;
+    int seg_len;
+    int P = plan_segments(U, N, di->sms, &seg_len);
+    p.seg_len = seg_len;
+    const size_t ws_need = segment_workspace_bytes(U, P, dk, dv);
+    if (P > 1 && (!workspace || ws_bytes < ws_need || !aligned16(workspace) ||
+                  (long)U * P * tc::NVS > (1L << 30))) {
+        P = 1;  // no room for the segment states: one pass over whole sequences
+        p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
+    }
     // With N = 0 no tile is ever copied; the maps then only need a valid base.
     const void* bq = N > 0 ? q : s_out;
     const void* bk = N > 0 ? k : s_out;
@@ -269,6 +316,29 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     if ((s = make_map(&mk, bk, dk, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mv, bv, dv, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mo, bo, dv, Nm, U, row, unit, 32, 1)) != LA_OK) return s;
+    if (P > 1) {
+        // segment split: (1) the K^T V sum of every segment but the last,
+        // (2) the state before every segment, (3) all segments from those states
+        float* seg_sums = reinterpret_cast<float*>(workspace);
+        float* starts = seg_sums + (size_t)U * (P - 1) * dk * dv;
+        tc::Params p1 = p;
+        p1.n_seg = P - 1;
+        p1.n_items = (int)(U * (P - 1) * tc::NVS);
+        p1.s0 = nullptr;
+        p1.s_out = seg_sums;
+        p1.s_out_per_seg = 1;
+        p1.state_only = 1;
+        tc::prefill_tc_kernel<<<std::min(p1.n_items, di->sms), tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv,
+                                                                                                   mo, p1);
+        if ((s = after_launch("prefill_tc (segment sums) launch")) != LA_OK) return s;
+        const long threads = U * (long)(dk * dv / 4);
+        const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
+        segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(seg_sums, s0, starts, U, P, dk * dv);
+        if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
+        p.n_seg = P;
+        p.n_items = (int)(U * P * tc::NVS);
+        p.seg_init = starts;
+    }
     const int grid = std::min(p.n_items, di->sms);
     tc::prefill_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
     return after_launch("prefill_tc launch");
@@ -341,6 +411,7 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
 
     tc::Params p{};
     p.mode = 1;
+    p.n_seg = 1;
     p.n_items = (int)((long)n_seq * H * tc::NVS);
     p.H = H;
     p.dv = dv;

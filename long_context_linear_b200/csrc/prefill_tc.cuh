@@ -100,18 +100,26 @@ struct Params {
     const float* s0;       // dense: [U][DK][dv] or null
     const float* pool;     // packed: [n_pool][H][DK][dv] or null
     const int* init_idx;   // packed: [n_seq] or null
-    float* s_out;          // [U or n_seq*H][DK][dv] or null
+    float* s_out;          // [U or n_seq*H or U*n_seg][DK][dv] or null
     __nv_bfloat16* o;      // output base, for direct stores of ragged tails
     int* status;           // device status word
+    // dense only: the sequence of each unit cut into n_seg segments of seg_len
+    // tokens (a multiple of C; the last one may be shorter)
+    int n_seg;
+    int seg_len;
+    const float* seg_init; // [U][n_seg][DK][dv]: state before each segment, or null (then s0)
+    int s_out_per_seg;     // 1: s_out holds the state after every segment, [U][n_seg][DK][dv]
+    int state_only;        // 1: only the state is computed (no Q, no outputs)
 };
 
 struct Item {
-    int t0;         // first token (packed: absolute row; dense: 0)
+    int t0;         // first token (packed: absolute row; dense: segment start)
     int len;        // tokens
     int c1, c2;     // TMA coordinates (dense: unit in c2; packed: head in c1)
     int vs;         // value slice
-    long state;     // index of the (unit | sequence*H + head) state
+    long state;     // index of the (unit | sequence*H + head | unit*n_seg + segment) state
     const float* init;  // initial state row block or null
+    bool write_state;   // the item's final state goes to s_out
 };
 
 __device__ __forceinline__ int item_index(int round, int cta, int grid) {
@@ -124,13 +132,16 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     Item it;
     it.vs = idx & (NVS - 1);
     if (p.mode == 0) {
-        const int u = idx / NVS;
-        it.t0 = 0;
-        it.len = p.N;
+        const int us = idx / NVS;  // unit * n_seg + segment
+        const int u = us / p.n_seg, sg = us - u * p.n_seg;
+        it.t0 = sg * p.seg_len;
+        it.len = min(p.seg_len, p.N - it.t0);
         it.c1 = 0;
         it.c2 = u;
-        it.state = u;
-        it.init = p.s0 ? p.s0 + (long)u * DK * p.dv : nullptr;
+        it.state = p.s_out_per_seg ? us : u;
+        it.init = p.seg_init ? p.seg_init + (long)us * DK * p.dv
+                             : ((sg == 0 && p.s0) ? p.s0 + (long)u * DK * p.dv : nullptr);
+        it.write_state = p.s_out_per_seg || sg == p.n_seg - 1;
     } else {
         const int hs = idx / NVS;   // sequence rank * H + head
         const int r = hs / p.H;
@@ -143,6 +154,7 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
         it.state = (long)seq * p.H + h;
         const int ii = p.init_idx ? p.init_idx[seq] : -1;
         it.init = (p.pool && ii >= 0) ? p.pool + ((long)ii * p.H + h) * DK * p.dv : nullptr;
+        it.write_state = true;
     }
     return it;
 }
@@ -230,12 +242,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         for (int i = 0; i < K_SLOTS; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 2);
+            mbar_init(&k_empty[i], p.state_only ? 1 : 2);
             mbar_init(&s_full[i], 4);
         }
         for (int i = 0; i < V_SLOTS; ++i) {
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 2);
+            mbar_init(&v_empty[i], p.state_only ? 1 : 2);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&p_full[i], 1);
@@ -279,21 +291,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int c = -PREFETCH; c < nc; ++c) {
                     const int cp = c + PREFETCH;
                     if (cp < nc) {
-                        const int y = p.mode == 0 ? cp * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + cp * C;
-                        tma_prefetch_3d(&map_q, 0, y, z);
-                        tma_prefetch_3d(&map_q, 64, y, z);
+                        const int y = p.mode == 0 ? it.t0 + cp * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + cp * C;
+                        if (!p.state_only) {
+                            tma_prefetch_3d(&map_q, 0, y, z);
+                            tma_prefetch_3d(&map_q, 64, y, z);
+                        }
                         tma_prefetch_3d(&map_k, 0, y, z);
                         tma_prefetch_3d(&map_k, 64, y, z);
                         tma_prefetch_3d(&map_v, DVS * it.vs, y, z);
                     }
                     if (c < 0) continue;
-                    const int y = p.mode == 0 ? c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
+                    const int y = p.mode == 0 ? it.t0 + c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
                     const int qs = g % Q_SLOTS, kq = g / Q_SLOTS;
-                    if (kq > 0 && !mbar_wait(&q_empty[qs], (kq - 1) & 1, abort, p.status)) { stop = true; break; }
-                    uint8_t* qb = sm + OFF_Q + qs * TILE_Q;
-                    mbar_arrive_expect_tx(&q_full[qs], TILE_Q);
-                    tma_load_3d(qb, &map_q, &q_full[qs], 0, y, z);
-                    tma_load_3d(qb + PANEL, &map_q, &q_full[qs], 64, y, z);
+                    if (!p.state_only) {
+                        if (kq > 0 && !mbar_wait(&q_empty[qs], (kq - 1) & 1, abort, p.status)) { stop = true; break; }
+                        uint8_t* qb = sm + OFF_Q + qs * TILE_Q;
+                        mbar_arrive_expect_tx(&q_full[qs], TILE_Q);
+                        tma_load_3d(qb, &map_q, &q_full[qs], 0, y, z);
+                        tma_load_3d(qb + PANEL, &map_q, &q_full[qs], 64, y, z);
+                    }
                     const int ks = g % K_SLOTS, kk_ = g / K_SLOTS;
                     if (kk_ > 0 && !mbar_wait(&k_empty[ks], (kk_ - 1) & 1, abort, p.status)) { stop = true; break; }
                     uint8_t* kb = sm + OFF_K + ks * TILE_K;
@@ -305,7 +321,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
             // make sure no copy into shared memory is still in flight at exit
             for (int x = (g >= Q_SLOTS ? g - Q_SLOTS : 0); x < g; ++x) {
-                drain_wait(&q_full[x % Q_SLOTS], (x / Q_SLOTS) & 1);
+                if (!p.state_only) drain_wait(&q_full[x % Q_SLOTS], (x / Q_SLOTS) & 1);
                 drain_wait(&k_full[x % K_SLOTS], (x / K_SLOTS) & 1);
             }
         }
@@ -320,7 +336,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const Item it = decode_item(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
-                    const int y = p.mode == 0 ? c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
+                    const int y = p.mode == 0 ? it.t0 + c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
                     const int vc = g % V_SLOTS, kv = g / V_SLOTS;
                     if (kv > 0 && !mbar_wait(&v_empty[vc], (kv - 1) & 1, abort, p.status)) { stop = true; break; }
                     mbar_arrive_expect_tx(&v_full[vc], PANEL);
@@ -336,7 +352,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // P V of chunk g, so its mask runs while P V and the next product are
         // queued.  TMEM written or read by other warps is ordered by
         // tcgen05.fence::after_thread_sync after the barrier.
-        if (lane == 0) {
+        if (lane == 0 && !p.state_only) {
             constexpr uint32_t id_f = idesc_bf16(128, C + DVS, 0, 0);  // Q [K ; S^T]^T
             constexpr uint32_t id_pv = idesc_bf16(128, DVS, 0, 1);     // P V (P from TMEM)
             const uint32_t sq = smem_u32(sm + OFF_Q), sk = smem_u32(sm + OFF_K), sv = smem_u32(sm + OFF_V);
@@ -439,46 +455,48 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         __syncwarp();
     } else if (warp < 6) {
-        // ------------------------------------------------------ mask warps
-        // Row t = 32 q4 + lane of P; 32-column piece pc holds keys 32 pc ...
-        // Pieces below the diagonal piece are kept whole, the diagonal piece
-        // keeps s <= t, pieces above it are zero.  bf16 piece pc goes to
-        // columns 16 pc .. 16 pc + 15, which only overlap fp32 pieces already read.
-        const int q4 = warp & 3;
-        int g = 0;
-        bool stop = false;
-        for (int r = 0; !stop; ++r) {
-            const int idx = item_index(r, cta, G);
-            if (idx >= p.n_items) break;
-            const int len = decode_item(p, idx).len;
-            for (int c0 = 0; c0 < len; c0 += C, ++g) {
-                const int b = g & 1;
-                if (!warp_wait(&p_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_PO_STRIDE * b;
+        if (!p.state_only) {
+            // ------------------------------------------------------ mask warps
+            // Row t = 32 q4 + lane of P; 32-column piece pc holds keys 32 pc ...
+            // Pieces below the diagonal piece are kept whole, the diagonal piece
+            // keeps s <= t, pieces above it are zero.  bf16 piece pc goes to
+            // columns 16 pc .. 16 pc + 15, which only overlap fp32 pieces already read.
+            const int q4 = warp & 3;
+            int g = 0;
+            bool stop = false;
+            for (int r = 0; !stop; ++r) {
+                const int idx = item_index(r, cta, G);
+                if (idx >= p.n_items) break;
+                const int len = decode_item(p, idx).len;
+                for (int c0 = 0; c0 < len; c0 += C, ++g) {
+                    const int b = g & 1;
+                    if (!warp_wait(&p_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_PO_STRIDE * b;
 #pragma unroll 1
-                for (int pc = 0; pc < 4; ++pc) {
-                    uint32_t pk[16];
-                    if (pc <= q4) {
-                        uint32_t v[32];
-                        tmem_ld32(ta + 32 * pc, v);
-                        tmem_wait_ld();
-                        const int keep = pc < q4 ? 31 : lane;  // last kept column within the piece
+                    for (int pc = 0; pc < 4; ++pc) {
+                        uint32_t pk[16];
+                        if (pc <= q4) {
+                            uint32_t v[32];
+                            tmem_ld32(ta + 32 * pc, v);
+                            tmem_wait_ld();
+                            const int keep = pc < q4 ? 31 : lane;  // last kept column within the piece
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(2 * i <= keep ? __uint_as_float(v[2 * i]) : 0.f,
-                                                2 * i + 1 <= keep ? __uint_as_float(v[2 * i + 1]) : 0.f);
-                    } else {
+                            for (int i = 0; i < 16; ++i)
+                                pk[i] = pack_bf16x2(2 * i <= keep ? __uint_as_float(v[2 * i]) : 0.f,
+                                                    2 * i + 1 <= keep ? __uint_as_float(v[2 * i + 1]) : 0.f);
+                        } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                        }
+                        tmem_st16(ta + 16 * pc, pk);
                     }
-                    tmem_st16(ta + 16 * pc, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    // the P V product of this chunk also needs V_c
+                    if (!warp_wait(&v_full[g % V_SLOTS], (g / V_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                    if (lane == 0) mbar_arrive(&p_ready[b]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                // the P V product of this chunk also needs V_c
-                if (!warp_wait(&v_full[g % V_SLOTS], (g / V_SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                if (lane == 0) mbar_arrive(&p_ready[b]);
             }
         }
     } else if (warp < 10) {
@@ -512,23 +530,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
                 // publish bf16(S_{c-1})^T next to K_c, once the slot's previous product is done
                 const int ks = g % K_SLOTS;
-                if (g >= K_SLOTS && !warp_wait(&k_empty[ks], ((g / K_SLOTS) - 1) & 1, abort, p.status)) { stop = true; break; }
-                uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
-                __nv_bfloat16* rowp[8];
+                if (!p.state_only) {
+                    if (g >= K_SLOTS && !warp_wait(&k_empty[ks], ((g / K_SLOTS) - 1) & 1, abort, p.status)) { stop = true; break; }
+                    uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
+                    __nv_bfloat16* rowp[8];
 #pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    rowp[m] = reinterpret_cast<__nv_bfloat16*>(base + ((colchunk ^ static_cast<uint32_t>(m)) << 4));
+                    for (int m = 0; m < 8; ++m)
+                        rowp[m] = reinterpret_cast<__nv_bfloat16*>(base + ((colchunk ^ static_cast<uint32_t>(m)) << 4));
 #pragma unroll
-                for (int j = 0; j < DVS; ++j) rowp[j & 7][j * 64] = __float2bfloat16_rn(S[j]);
-                fence_proxy_async_smem();
-                // the [P|O] product of this chunk also needs Q_c, K_c and the O
-                // buffer it writes (last used by chunk c - 2) drained
-                if (!warp_wait(&q_full[g % Q_SLOTS], (g / Q_SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                if (!warp_wait(&k_full[ks], (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                if (g >= 2 && !warp_wait(&o_empty[g & 1], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                tc_fence_before();
-                if (lane == 0) mbar_arrive(&s_full[ks]);
+                    for (int j = 0; j < DVS; ++j) rowp[j & 7][j * 64] = __float2bfloat16_rn(S[j]);
+                    fence_proxy_async_smem();
+                    // the [P|O] product of this chunk also needs Q_c, K_c and the O
+                    // buffer it writes (last used by chunk c - 2) drained
+                    if (!warp_wait(&q_full[g % Q_SLOTS], (g / Q_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                    if (!warp_wait(&k_full[ks], (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                    if (g >= 2 && !warp_wait(&o_empty[g & 1], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    tc_fence_before();
+                    if (lane == 0) mbar_arrive(&s_full[ks]);
+                }
                 // absorb dS_c
                 const int b = g & 1;
                 if (!warp_wait(&ds_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
@@ -546,7 +566,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (lane == 0) mbar_arrive(&ds_empty[b]);
             }
             if (stop) break;
-            if (p.s_out) {
+            if (p.s_out && it.write_state) {
                 float4* dst = reinterpret_cast<float4*>(p.s_out + (it.state * DK + i) * p.dv + DVS * it.vs);
 #pragma unroll
                 for (int j = 0; j < DVS / 4; ++j)
@@ -554,69 +574,71 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
         }
     } else if (warp < 14) {
-        // ------------------------------------------------------ output warps
-        const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;
-        uint8_t* stg = sm + OFF_OST + q4 * OST_WARP;  // this warp's 32 staging rows
-        int g = 0;
-        bool stop = false;
-        for (int r = 0; !stop; ++r) {
-            const int idx = item_index(r, cta, G);
-            if (idx >= p.n_items) break;
-            const Item it = decode_item(p, idx);
-            for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
-                const int b = g & 1;
-                if (!warp_wait(&o_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
-                tc_fence_after();
-                const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_PO_STRIDE * b + TM_O_OFF;
-                uint32_t hp[32];
-                {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(ta, v0);
-                    tmem_ld32(ta + 32, v1);
-                    tmem_wait_ld();
+        if (!p.state_only) {
+            // ------------------------------------------------------ output warps
+            const int q4 = warp & 3;
+            const int row = q4 * 32 + lane;
+            uint8_t* stg = sm + OFF_OST + q4 * OST_WARP;  // this warp's 32 staging rows
+            int g = 0;
+            bool stop = false;
+            for (int r = 0; !stop; ++r) {
+                const int idx = item_index(r, cta, G);
+                if (idx >= p.n_items) break;
+                const Item it = decode_item(p, idx);
+                for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
+                    const int b = g & 1;
+                    if (!warp_wait(&o_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t ta = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_PO_STRIDE * b + TM_O_OFF;
+                    uint32_t hp[32];
+                    {
+                        uint32_t v0[32], v1[32];
+                        tmem_ld32(ta, v0);
+                        tmem_ld32(ta + 32, v1);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        hp[e] = pack_bf16x2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
-                        hp[16 + e] = pack_bf16x2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
+                        for (int e = 0; e < 16; ++e) {
+                            hp[e] = pack_bf16x2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
+                            hp[16 + e] = pack_bf16x2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
+                        }
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&o_empty[b]);
-                const int rows = it.len - c0;
-                if (q4 * 32 >= rows) {
-                    // this warp's rows all lie past the end of the sequence
-                } else if (p.mode == 0 || q4 * 32 + 32 <= rows) {
-                    // each warp stages its 32 rows and stores them with one TMA copy
-                    // (a dense tensor clips rows past N itself)
-                    if (lane == 0) bulk_wait_read<0>();
+                    tc_fence_before();
                     __syncwarp();
-                    const uint32_t sa = smem_u32(stg) + static_cast<uint32_t>(lane) * 128u;
+                    if (lane == 0) mbar_arrive(&o_empty[b]);
+                    const int rows = it.len - c0;
+                    if (q4 * 32 >= rows) {
+                        // this warp's rows all lie past the end of the sequence
+                    } else if (p.mode == 0 || q4 * 32 + 32 <= rows) {
+                        // each warp stages its 32 rows and stores them with one TMA copy
+                        // (a dense tensor clips rows past N itself)
+                        if (lane == 0) bulk_wait_read<0>();
+                        __syncwarp();
+                        const uint32_t sa = smem_u32(stg) + static_cast<uint32_t>(lane) * 128u;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        st_shared_v4(sa + ((static_cast<uint32_t>(ch) ^ (row & 7)) << 4), hp[4 * ch], hp[4 * ch + 1],
-                                     hp[4 * ch + 2], hp[4 * ch + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (p.mode == 0) tma_store_3d(&map_o, stg, DVS * it.vs, c0 + q4 * 32, it.c2);
-                        else tma_store_3d(&map_o, stg, DVS * it.vs, it.c1, it.t0 + c0 + q4 * 32);
-                        bulk_commit();
+                        for (int ch = 0; ch < 8; ++ch)
+                            st_shared_v4(sa + ((static_cast<uint32_t>(ch) ^ (row & 7)) << 4), hp[4 * ch], hp[4 * ch + 1],
+                                         hp[4 * ch + 2], hp[4 * ch + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (p.mode == 0) tma_store_3d(&map_o, stg, DVS * it.vs, it.t0 + c0 + q4 * 32, it.c2);
+                            else tma_store_3d(&map_o, stg, DVS * it.vs, it.c1, it.t0 + c0 + q4 * 32);
+                            bulk_commit();
+                        }
+                    } else if (row < rows) {
+                        // ragged tail of a packed sequence (the next rows belong to
+                        // another sequence): plain row stores
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            p.o + ((long)(it.t0 + c0 + row) * p.H + it.c1) * p.dv + DVS * it.vs);
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            dst[ch] = make_uint4(hp[4 * ch], hp[4 * ch + 1], hp[4 * ch + 2], hp[4 * ch + 3]);
                     }
-                } else if (row < rows) {
-                    // ragged tail of a packed sequence (the next rows belong to
-                    // another sequence): plain row stores
-                    uint4* dst = reinterpret_cast<uint4*>(
-                        p.o + ((long)(it.t0 + c0 + row) * p.H + it.c1) * p.dv + DVS * it.vs);
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        dst[ch] = make_uint4(hp[4 * ch], hp[4 * ch + 1], hp[4 * ch + 2], hp[4 * ch + 3]);
                 }
             }
+            if (lane == 0) bulk_wait<0>();
+            __syncwarp();
         }
-        if (lane == 0) bulk_wait<0>();
-        __syncwarp();
     }
 
     tc_fence_before();

@@ -1,0 +1,109 @@
+"""Segment split of the dense tensor-core prefill (few units, long sequences).
+
+The sequence of each unit is cut into segments of whole chunks; a state-only
+pass sums K^T V per segment, a prefix kernel forms the state before every
+segment, and the main pass runs all segments from those states.  The result is
+the same recurrence (page "MiniMax-M1で理解する…", section
+"線形アテンションの数学的基礎"), so every case is checked against the fp64
+oracle, and inputs whose every partial sum is an exact integer must agree bit
+for bit whatever the segment count.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.parity import assert_guard_intact, assert_out, assert_state, guarded, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def la():
+    import long_context_linear_b200 as la
+    return la
+
+
+def _run(la, q, k, v, s0=None):
+    B, H, N, d = q.shape
+    out, full_o = guarded((B, H, N, d), q.dtype)
+    s_out, full_s = guarded((B, H, d, d), torch.float32)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), None if s0 is None else s0.cuda(), out=out, s_out=s_out)
+    torch.cuda.synchronize()
+    assert_guard_intact(full_o, out.numel())
+    assert_guard_intact(full_s, s_out.numel())
+    assert la.device_status() == 0
+    return o.cpu(), s.cpu()
+
+
+def _state(B, H, d, seed, L=300):
+    return synth.outer_product_state(B * H, d, d, [L] * (B * H), seed=seed).view(B, H, d, d)
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 1, 20000), (1, 2, 9000), (2, 1, 4096 + 77)])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_auto_segments_match_oracle(la, oracle_mod, B, H, N, with_s0):
+    assert la.prefill_workspace_size(B, H, N, 128, torch.bfloat16) > 0, "shape should be split"
+    q, k, v = synth.dense(B, H, N, 128, "bf16", seed=7 * N + B + H)
+    s0 = _state(B, H, 128, seed=N) if with_s0 else None
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.bfloat16, 2)
+    assert_state(s, rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["1", "2", "3", "7", "40"])
+def test_forced_segment_counts(la, oracle_mod, monkeypatch, segments):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v = synth.dense(1, 2, 5000, 128, "bf16", seed=11)
+    s0 = _state(1, 2, 128, seed=12)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.bfloat16, 2)
+    assert_state(s, rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["1", "4", "9"])
+def test_segments_integer_inputs_bit_exact(la, oracle_mod, monkeypatch, segments):
+    """Inputs in {-1,0,1} and an integer S0: every product and partial sum is an
+    exact integer (|S| stays well inside the range where bf16(S) is exact), so
+    the split must not change a single bit."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N, d = 1, 2, 1500, 128
+    q = synth.integer_valued((B, H, N, d), seed=21, dtype=torch.bfloat16)
+    k = synth.integer_valued((B, H, N, d), seed=22, dtype=torch.bfloat16)
+    v = synth.integer_valued((B, H, N, d), seed=23, dtype=torch.bfloat16)
+    s0 = synth.integer_valued((B, H, d, d), seed=24, lo=-20, hi=20, dtype=torch.float32)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert torch.equal(o, torch.from_numpy(ro).to(torch.bfloat16))
+    np.testing.assert_array_equal(to64(s), rs)
+
+
+def test_without_workspace_runs_unsplit(la, oracle_mod):
+    """A caller that passes no workspace gets the one-pass sweep (same result)."""
+    B, H, N, d = 1, 1, 6000, 128
+    assert la.prefill_workspace_size(B, H, N, d, torch.bfloat16) > 0
+    q, k, v = (x.cuda() for x in synth.dense(B, H, N, d, "bf16", seed=31))
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device="cuda")
+    st = la.lib.la_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, s.data_ptr(), B, H, N, d,
+                           d, 0, 0, None, 0, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q.cpu(), k.cpu(), v.cpu())
+    assert_out(o.cpu(), ro, torch.bfloat16, 2)
+    assert_state(s.cpu(), rs, 2)
+
+
+def test_workspace_size_follows_the_plan(la):
+    # 64 heads fill the GPU: no split, no workspace
+    assert la.prefill_workspace_size(1, 64, 131072, 128, torch.bfloat16) == 0
+    # short sequences are never split
+    assert la.prefill_workspace_size(1, 1, 512, 128, torch.bfloat16) == 0
+    # one head over 64K tokens: (2P - 1) fp32 states of 128 x 128
+    n = la.prefill_workspace_size(1, 1, 65536, 128, torch.bfloat16)
+    assert n > 0 and n % (128 * 128 * 4) == 0 and (n // (128 * 128 * 4)) % 2 == 1
