@@ -279,7 +279,7 @@ def run_headline(args, dist: Dist, pk, sampler: ClockSampler):
     return res, sample
 
 
-def run_decode(args, dist: Dist, pk):
+def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
     import long_context_linear_b200 as la
     import synth
     c = DECODE
@@ -292,7 +292,7 @@ def run_decode(args, dist: Dist, pk):
     grp = 2048
     for u0 in range(0, U, grp):
         S[u0:u0 + grp] = synth.outer_product_state(min(grp, U - u0), d, d, L[u0:u0 + grp], seed=7 + u0, device=dev)
-    S = S.view(B, H, d, d)
+    S = S.view(B, H, d, d).to(state_dtype)
     qs, ks, vs = synth.qkv((steps, B, H, d), d, "bf16", seed=43 + dist.rank, device=dev)
     os_ = torch.empty_like(vs)
     stream = torch.cuda.current_stream(dev)
@@ -307,11 +307,13 @@ def run_decode(args, dist: Dist, pk):
     total_ms, per = timed_launches(step, steps, max(3, args.warmup), dist, stream)
     total_ms = dist.max(total_ms)
     ms_step = total_ms / steps
-    bytes_step = 2.0 * U * d * d * 4 + 4.0 * U * d * 2
+    esz = torch.empty(0, dtype=state_dtype).element_size()
+    bytes_step = 2.0 * U * d * d * esz + 4.0 * U * d * 2
     gbs = bytes_step / (ms_step / 1e3) / 1e9
     del S, qs, ks, vs, os_
     torch.cuda.empty_cache()
-    return dict(workload="decode B=256 H=64 d=128 bf16 q/k/v, fp32 state, 1024 consecutive steps",
+    name = {torch.float32: "fp32", torch.bfloat16: "bf16", torch.float16: "fp16"}[state_dtype]
+    return dict(workload=f"decode B=256 H=64 d=128 bf16 q/k/v, {name} state, 1024 consecutive steps",
                 hbm_gbs=gbs, peak_gbs=pk["hbm"], frac=gbs / pk["hbm"], ms_per_step=ms_step,
                 bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
 
@@ -508,6 +510,9 @@ def main():
     extras = {}
     if not args.no_extras:
         extras["decode"] = run_decode(args, dist, pk)
+        # state stored in bf16 / fp16, updated in fp32 (the low-precision storage study)
+        extras["decode_bf16_state"] = run_decode(args, dist, pk, torch.bfloat16)
+        extras["decode_fp16_state"] = run_decode(args, dist, pk, torch.float16)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["few_heads"] = run_few_heads(args, dist, pk)

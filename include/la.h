@@ -63,6 +63,9 @@ typedef enum {
 
 typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
 
+/* Storage format of a decode state (see la_decode_step_state). */
+typedef enum { LA_STATE_FP32 = 0, LA_STATE_BF16 = 1, LA_STATE_FP16 = 2 } la_state_dtype;
+
 /* Same type as cudaStream_t (an opaque CUDA stream handle). */
 typedef struct CUstream_st* la_stream_t;
 
@@ -134,6 +137,22 @@ LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v, 
  */
 LA_API la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S,
                          int B, int H, int dk, int dv, la_dtype dt, la_stream_t stream);
+
+/*
+ * la_decode_step with the state stored in a chosen format, for the study of
+ * low-precision state storage that page "MiniMax: «Почему M2 …»", section 4,
+ * and page "ノーフリーランチ：MiniMax M2が高効率アテンション機構を解体",
+ * infrastructure section, warn about (the state is rewritten at every token,
+ * so its rounding errors accumulate).
+ *   S: [B, H, d, d] in `sdt` (fp32, bf16 or fp16), updated IN PLACE.
+ *   Each element is updated in fp32 as RN_fp32(S + k_i v_j) (one fused
+ *   multiply-add) and rounded to `sdt` to nearest even; o = q S uses the
+ *   stored, rounded state.  LA_STATE_FP32 is exactly la_decode_step.
+ *   Low-precision storage needs bf16 q, k, v (LA_ERR_UNSUPPORTED otherwise).
+ */
+LA_API la_status la_decode_step_state(const void* q, const void* k, const void* v, void* o, void* S,
+                                      int B, int H, int dk, int dv, la_dtype dt, la_state_dtype sdt,
+                                      la_stream_t stream);
 
 /*
  * Reads the device status word of the current device (synchronizes the

@@ -172,15 +172,23 @@ def prefill_varlen_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu
                    "la_prefill_varlen_noalloc")
 
 
+_STATE_DT = {torch.float32: _abi.LA_STATE_FP32, torch.bfloat16: _abi.LA_STATE_BF16,
+             torch.float16: _abi.LA_STATE_FP16}
+
+
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token per (batch, head): S <- S + k (x) v in place, returns o = q S.
 
-    q, k, v: [B, H, d]; S: fp32 [B, H, d, d].
+    q, k, v: [B, H, d]; S: [B, H, d, d] in fp32, or in bf16 / fp16 (state
+    stored in low precision, updated in fp32 and rounded to nearest even;
+    needs bf16 q, k, v).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype, q.device)
-    _need(S, "S", torch.float32, q.device)
+    if S.dtype not in _STATE_DT:
+        raise TypeError(f"S must be float32, bfloat16 or float16, got {S.dtype}")
+    _need(S, "S", S.dtype, q.device)
     if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
         raise ValueError("q, k must be [B, H, dk] and v [B, H, dv]")
     B, H, dk = q.shape
@@ -191,8 +199,9 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tens
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _need(out, "out", q.dtype, q.device)
     with torch.cuda.device(q.device):
-        _abi.check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, dk, dv,
-                                      _dtype_code(q), _stream(q.device)), "la_decode_step")
+        _abi.check(lib.la_decode_step_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, dk, dv,
+                                            _dtype_code(q), _STATE_DT[S.dtype], _stream(q.device)),
+                   "la_decode_step_state")
     return out
 
 

@@ -18,6 +18,9 @@ LA_ERR_CUDA = 3
 LA_ERR_TIMEOUT = 4
 LA_BF16 = 0
 LA_FP32 = 1
+LA_STATE_FP32 = 0
+LA_STATE_BF16 = 1
+LA_STATE_FP16 = 2
 
 # name -> (restype, argtypes), mirroring include/la.h
 _vp = ctypes.c_void_p
@@ -33,6 +36,7 @@ SIGNATURES = {
     "la_prefill_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i,
                                _vp, _sz, _vp]),
     "la_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_step_state": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
     "la_selftest_wait_timeout": (_i, [_i, _vp]),
     "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),

@@ -4,12 +4,19 @@
 // "MiniMax-M1で理解する…", section "線形アテンションの数学的基礎", one token at a
 // time; page "MiniMax: «Почему M2 …»", section 4, notes this is a small state
 // matrix that is read and written on every step).  One CTA streams one d x d
-// fp32 state once: every thread owns 4 consecutive value columns of D/RS rows,
-// loads them with 16-byte streaming loads (all loads issued before any use),
-// updates, stores them back, and accumulates its share of o; partial sums are
-// reduced across row slots in shared memory.
+// state once: every thread owns one 16-byte vector of E consecutive value
+// columns in each of D/RS rows, loads them with streaming loads (all loads
+// issued before any use), updates, stores them back, and accumulates its share
+// of o; partial sums are reduced across row slots in shared memory.
+//
+// The state may be stored in fp32, bf16 or fp16 (the low-precision state
+// storage the same section warns about).  The update is always computed in
+// fp32: S_new = RN_fp32(S_stored + k_i v_j) (one fused multiply-add, the
+// product of two bf16 inputs being exact in fp32), then rounded to the storage
+// format to nearest even; o uses the stored (rounded) state.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace lcl {
 namespace dec {
@@ -21,55 +28,115 @@ __device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat1
 __device__ __forceinline__ void st_f(float* p, float x) { *p = x; }
 __device__ __forceinline__ void st_f(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
-template <typename T, int D>
+// E values of one 16-byte state vector <-> fp32
+template <typename SS> struct Vec;
+template <> struct Vec<float> {
+    static constexpr int E = 4;
+    __device__ __forceinline__ static void unpack(const uint4& r, float (&f)[4]) {
+        f[0] = __uint_as_float(r.x); f[1] = __uint_as_float(r.y); f[2] = __uint_as_float(r.z); f[3] = __uint_as_float(r.w);
+    }
+    // rounds f to the storage format in place and packs it
+    __device__ __forceinline__ static uint4 pack(float (&f)[4]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+template <> struct Vec<__nv_bfloat16> {
+    static constexpr int E = 8;
+    __device__ __forceinline__ static void unpack(const uint4& r, float (&f)[8]) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(float (&f)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h);
+            f[2 * i] = __low2float(h);
+            f[2 * i + 1] = __high2float(h);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+template <> struct Vec<__half> {
+    static constexpr int E = 8;
+    __device__ __forceinline__ static void unpack(const uint4& r, float (&f)[8]) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+            f[2 * i] = __low2float(h);
+            f[2 * i + 1] = __high2float(h);
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(float (&f)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h);
+            f[2 * i] = __low2float(h);
+            f[2 * i + 1] = __high2float(h);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <typename T, typename SS, int D>
 __global__ void __launch_bounds__(NUM_THREADS)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
-                   float* __restrict__ S) {
-    constexpr int TPR = D / 4;             // threads per row
+                   SS* __restrict__ S) {
+    constexpr int E = Vec<SS>::E;          // state values per 16-byte vector
+    constexpr int TPR = D / E;             // threads per row
     constexpr int RS = NUM_THREADS / TPR;  // row slots
     constexpr int RPT = D / RS;            // rows per thread
     __shared__ float qs[D], ks[D], vs[D];
-    __shared__ float4 red[RS][TPR];
+    __shared__ float red[RS][D];
 
     const long u = blockIdx.x;
     const int tid = threadIdx.x;
-    const int c4 = tid % TPR;
+    const int cv = tid % TPR;
     const int slot = tid / TPR;
-    float4* Su = reinterpret_cast<float4*>(S + u * D * D);
+    uint4* Su = reinterpret_cast<uint4*>(S + u * D * D);
 
-    float4 x[RPT];
+    uint4 x[RPT];
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) x[m] = __ldcs(&Su[(slot + m * RS) * TPR + c4]);
+    for (int m = 0; m < RPT; ++m) x[m] = __ldcs(&Su[(slot + m * RS) * TPR + cv]);
     if (tid < D) {
         qs[tid] = ld_f(q + u * D + tid);
         ks[tid] = ld_f(k + u * D + tid);
         vs[tid] = ld_f(v + u * D + tid);
     }
     __syncthreads();
-    const float4 vj = make_float4(vs[4 * c4], vs[4 * c4 + 1], vs[4 * c4 + 2], vs[4 * c4 + 3]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float vj[E], acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        vj[e] = vs[E * cv + e];
+        acc[e] = 0.f;
+    }
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
         const int i = slot + m * RS;
         const float ki = ks[i], qi = qs[i];
-        float4 y = x[m];
-        y.x = fmaf(ki, vj.x, y.x);
-        y.y = fmaf(ki, vj.y, y.y);
-        y.z = fmaf(ki, vj.z, y.z);
-        y.w = fmaf(ki, vj.w, y.w);
-        __stcs(&Su[i * TPR + c4], y);
-        acc.x = fmaf(qi, y.x, acc.x);
-        acc.y = fmaf(qi, y.y, acc.y);
-        acc.z = fmaf(qi, y.z, acc.z);
-        acc.w = fmaf(qi, y.w, acc.w);
+        float y[E];
+        Vec<SS>::unpack(x[m], y);
+#pragma unroll
+        for (int e = 0; e < E; ++e) y[e] = fmaf(ki, vj[e], y[e]);
+        __stcs(&Su[i * TPR + cv], Vec<SS>::pack(y));
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(qi, y[e], acc[e]);
     }
-    red[slot][c4] = acc;
+#pragma unroll
+    for (int e = 0; e < E; ++e) red[slot][E * cv + e] = acc[e];
     __syncthreads();
     if (tid < D) {
-        const float* rf = reinterpret_cast<const float*>(&red[0][0]);
         float sum = 0.f;
 #pragma unroll
-        for (int s = 0; s < RS; ++s) sum += rf[s * D + tid];
+        for (int s = 0; s < RS; ++s) sum += red[s][tid];
         st_f(o + u * D + tid, sum);
     }
 }

@@ -195,6 +195,20 @@ la_status launch_simt(int d, int chunk, int grid, const void* q, const void* k, 
 }  // namespace
 }  // namespace lcl
 
+namespace lcl {
+namespace {
+template <typename T, typename SS>
+void launch_decode(int dk, int grid, const void* q, const void* k, const void* v, void* o, void* S, cudaStream_t st) {
+    if (dk == 128)
+        dec::decode_step_kernel<T, SS, 128><<<grid, dec::NUM_THREADS, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S);
+    else
+        dec::decode_step_kernel<T, SS, 64><<<grid, dec::NUM_THREADS, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S);
+}
+}  // namespace
+}  // namespace lcl
+
 using namespace lcl;
 
 extern "C" {
@@ -435,11 +449,15 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
     return after_launch("prefill_tc (varlen) launch");
 }
 
-la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S, int B, int H, int dk,
-                         int dv, la_dtype dt, la_stream_t stream) {
+la_status la_decode_step_state(const void* q, const void* k, const void* v, void* o, void* S, int B, int H, int dk,
+                               int dv, la_dtype dt, la_state_dtype sdt, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if (sdt != LA_STATE_FP32 && sdt != LA_STATE_BF16 && sdt != LA_STATE_FP16)
+        return fail(LA_ERR_INVALID_ARG, "unknown state dtype %d", (int)sdt);
+    if (sdt != LA_STATE_FP32 && dt != LA_BF16)
+        return fail(LA_ERR_UNSUPPORTED, "a bf16 or fp16 state needs bf16 q, k, v");
     if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
     const long U = (long)B * H;
     if (U == 0) return LA_OK;
@@ -451,16 +469,21 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o, f
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int grid = (int)U;
-    if (dt == LA_BF16) {
-        using T = __nv_bfloat16;
-        if (dk == 128) dec::decode_step_kernel<T, 128><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
-        else dec::decode_step_kernel<T, 64><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+    if (dt == LA_FP32) {
+        launch_decode<float, float>(dk, grid, q, k, v, o, S, st);
+    } else if (sdt == LA_STATE_FP32) {
+        launch_decode<__nv_bfloat16, float>(dk, grid, q, k, v, o, S, st);
+    } else if (sdt == LA_STATE_BF16) {
+        launch_decode<__nv_bfloat16, __nv_bfloat16>(dk, grid, q, k, v, o, S, st);
     } else {
-        using T = float;
-        if (dk == 128) dec::decode_step_kernel<T, 128><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
-        else dec::decode_step_kernel<T, 64><<<grid, dec::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S);
+        launch_decode<__nv_bfloat16, __half>(dk, grid, q, k, v, o, S, st);
     }
     return after_launch("decode_step launch");
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S, int B, int H, int dk,
+                         int dv, la_dtype dt, la_stream_t stream) {
+    return la_decode_step_state(q, k, v, o, S, B, H, dk, dv, dt, LA_STATE_FP32, stream);
 }
 
 namespace lcl {

@@ -123,6 +123,22 @@ def test_decode_rejects_bad_arguments(lib, kw, status):
     assert _decode(lib, **kw) == status
 
 
+def _decode_state(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, dk=128, dv=128, dt=0, sdt=1, stream=None)
+    a.update(kw)
+    return lib.la_decode_step_state(a["q"], a["k"], a["v"], a["o"], a["S"], a["B"], a["H"], a["dk"], a["dv"],
+                                    a["dt"], a["sdt"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(sdt=3), 1), (dict(sdt=-1), 1),   # unknown storage format
+    (dict(dt=1, sdt=1), 2),                # a bf16 state needs bf16 inputs
+    (dict(dt=1, sdt=2), 2),                # ... as does an fp16 state
+    (dict(S=None), 1), (dict(S=FAKE + 8), 1), (dict(B=-1), 1), (dict(dk=64, dv=128), 2)])
+def test_decode_state_rejects_bad_arguments(lib, kw, status):
+    assert _decode_state(lib, **kw) == status
+
+
 def test_device_status_null(lib):
     assert lib.la_device_status(None, 0) == 1
 

@@ -274,3 +274,71 @@ def test_pins_reject_planted_mistakes(mutant):
     ob, sb = _brute(qr, kr, vr, sr)
     brute_ok = _rel(om, ob) < 1e-12 and _rel(sm, sb) < 1e-12
     assert not (fixture_ok and brute_ok)
+
+
+# ------------------------------------------------- low-precision state storage
+# Pins of oracle/lowp.py against the definitions of the formats and of the
+# recurrence, not against itself.
+
+def test_lowp_bf16_rounding_follows_the_format_definition():
+    """bfloat16 keeps 8 significant bits; halfway cases go to the even mantissa."""
+    from oracle import lowp
+    x = np.array([1.0, 1 + 2**-8, 1 + 3 * 2**-8, 1 + 2**-8 + 2**-20, -(1 + 2**-8), 3.0, 255.0, 257.0, 259.0],
+                 dtype=np.float32)
+    want = np.array([1.0, 1.0, 1 + 2**-6, 1 + 2**-7, -1.0, 3.0, 255.0, 256.0, 260.0], dtype=np.float32)
+    np.testing.assert_array_equal(lowp.round_bf16(x), want)
+
+
+def test_lowp_fp16_rounding_follows_the_format_definition():
+    """binary16 keeps 11 significant bits, max 65504, smallest subnormal 2^-24."""
+    from oracle import lowp
+    x = np.array([1 + 2**-11, 1 + 3 * 2**-11, 65504.0, 2.0**-24, 2049.0, 2051.0], dtype=np.float32)
+    want = np.array([1.0, 1 + 2**-9, 65504.0, 2.0**-24, 2048.0, 2052.0], dtype=np.float32)
+    np.testing.assert_array_equal(lowp.round_fp16(x), want)
+
+
+@pytest.mark.parametrize("fmt", ["fp32", "bf16", "fp16"])
+def test_lowp_decode_is_exact_where_the_format_holds_every_value(oracle_mod, fmt):
+    """Integer inputs with |S| <= 64: every product, sum and stored value is
+    exact in all three formats, so 20 low-precision steps equal the fp64
+    recurrence bit for bit."""
+    from oracle import lowp
+    rng = np.random.default_rng(3)
+    U, d, T = 3, 16, 20
+    q, k, v = (rng.integers(-1, 2, (T, U, d)).astype(np.float64) for _ in range(3))
+    S = rng.integers(-30, 31, (U, d, d)).astype(np.float64)
+    S_exact, S_low = S.copy(), S.astype(np.float32)
+    for t in range(T):
+        o_ref, S_exact = oracle_mod.decode(q[t], k[t], v[t], S_exact)
+        o, S_low = lowp.decode_lowp(q[t], k[t], v[t], S_low, fmt)
+        np.testing.assert_array_equal(o, o_ref)
+        np.testing.assert_array_equal(S_low.astype(np.float64), S_exact)
+
+
+def test_lowp_decode_loses_updates_below_half_an_ulp():
+    """The storage effect the pages warn about, in closed form: a state entry of
+    256 with updates of +0.5 never moves in bf16 (ulp 2 at 256), moves by
+    exactly 0.5 per step in fp16 (ulp 0.25) and in fp32."""
+    from oracle import lowp
+    q = np.zeros(1)
+    k, v = np.ones(1), np.full(1, 0.5)
+    for fmt, want in (("bf16", 256.0), ("fp16", 261.0), ("fp32", 261.0)):
+        S = np.full((1, 1), 256.0, dtype=np.float32)
+        for _ in range(10):
+            _, S = lowp.decode_lowp(q, k, v, S, fmt)
+        assert S[0, 0] == want, (fmt, S[0, 0])
+
+
+def test_lowp_decode_fp32_tracks_the_fp64_recurrence(oracle_mod):
+    from oracle import lowp
+    rng = np.random.default_rng(5)
+    U, d, T = 2, 32, 50
+    q, k, v = (rng.standard_normal((T, U, d)) / np.sqrt(d) for _ in range(3))
+    q, k, v = (x.astype(np.float32).astype(np.float64) for x in (q, k, v))
+    S = (rng.standard_normal((U, d, d))).astype(np.float32)
+    S64 = S.astype(np.float64)
+    for t in range(T):
+        o_ref, S64 = oracle_mod.decode(q[t], k[t], v[t], S64)
+        o, S = lowp.decode_lowp(q[t], k[t], v[t], S, "fp32")
+    assert _rel(S.astype(np.float64), S64) < 1e-6
+    assert _rel(o, o_ref) < 1e-6
