@@ -318,6 +318,57 @@ def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
                 bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
 
 
+def run_speculative(args, dist: Dist, pk, m: int = 4):
+    """Decode B=256, H=64 with m draft tokens per step: one verify and one
+    commit of all m drafts, against m plain decode steps (same states)."""
+    import long_context_linear_b200 as la
+    import synth
+    c = DECODE
+    B, H, d = c["B"], c["H"], c["d"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    U = B * H
+    L_seq = synth.lengths(B, c["L_lo"], c["L_hi"], seed=41 + dist.rank)
+    L = [L_seq[u // H] for u in range(U)]
+    S = torch.empty(U, d, d, dtype=torch.float32, device=dev)
+    for u0 in range(0, U, 2048):
+        S[u0:u0 + 2048] = synth.outer_product_state(min(2048, U - u0), d, d, L[u0:u0 + 2048], seed=7 + u0, device=dev)
+    S = S.view(B, H, d, d)
+    rounds = 64
+    q, k, v = synth.qkv((rounds, B, H, m, d), d, "bf16", seed=47 + dist.rank, device=dev)
+    acc = torch.full((B,), m, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    it = [0]
+
+    def spec():
+        r = it[0] % rounds
+        la.decode_verify(q[r], k[r], v[r], S)
+        la.decode_commit(k[r], v[r], S, acc)
+        it[0] += 1
+
+    total_ms, _ = timed_launches(spec, rounds, max(3, args.warmup), dist, stream)
+    ms_spec = dist.max(total_ms) / rounds
+    qs, ks, vs = (x.permute(0, 3, 1, 2, 4).contiguous() for x in (q, k, v))  # [rounds, m, B, H, d]
+    it[0] = 0
+
+    def steps():
+        r = it[0] % rounds
+        for t in range(m):
+            la.decode_step(qs[r, t], ks[r, t], vs[r, t], S)
+        it[0] += 1
+
+    total_ms, _ = timed_launches(steps, rounds, max(3, args.warmup), dist, stream)
+    ms_steps = dist.max(total_ms) / rounds
+    bytes_spec = 3.0 * U * d * d * 4 + 4.0 * U * m * d * 2
+    del S, q, k, v, qs, ks, vs
+    torch.cuda.empty_cache()
+    return dict(workload=f"speculative decode B=256 H=64 d=128 bf16, fp32 state, m={m} drafts all accepted",
+                ms_verify_commit=ms_spec, ms_m_decode_steps=ms_steps,
+                tokens_per_s=B * m * dist.world / (ms_spec / 1e3),
+                tokens_per_s_decode_steps=B * m * dist.world / (ms_steps / 1e3),
+                hbm_gbs=bytes_spec / (ms_spec / 1e3) / 1e9, frac=bytes_spec / (ms_spec / 1e3) / 1e9 / pk["hbm"],
+                rounds=rounds)
+
+
 def run_varlen(args, dist: Dist, pk):
     import long_context_linear_b200 as la
     import synth
@@ -513,6 +564,7 @@ def main():
         # state stored in bf16 / fp16, updated in fp32 (the low-precision storage study)
         extras["decode_bf16_state"] = run_decode(args, dist, pk, torch.bfloat16)
         extras["decode_fp16_state"] = run_decode(args, dist, pk, torch.float16)
+        extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["few_heads"] = run_few_heads(args, dist, pk)

@@ -155,6 +155,26 @@ LA_API la_status la_decode_step_state(const void* q, const void* k, const void* 
                                       la_stream_t stream);
 
 /*
+ * Speculative decoding over m draft tokens per sequence (1 <= m <= 16): the
+ * state of a recurrent layer cannot be truncated after the fact (page
+ * "MiniMax: «Почему M2 …»", section 4), so verifying drafts and advancing the
+ * state are two calls.
+ *
+ * la_decode_verify: o_t = q_t S_t for every draft t = 1..m, where
+ *   S_t = S + sum_{s<=t} k_s (x) v_s; S itself is only read.
+ *   q, k : [B, H, m, d], v, o : [B, H, m, d]  dtype `dt`;  S : [B, H, d, d] fp32.
+ * la_decode_commit: S <- S + sum_{t < accepted[b]} k_t (x) v_t, IN PLACE, for
+ *   every head of sequence b; accepted: int32 device [B], values outside
+ *   [0, m] are clamped (checked on the host under LA_VALIDATE=1).  The
+ *   committed state is bit-identical to accepted[b] calls of la_decode_step.
+ * Each call reads the state once (commit also writes it back).
+ */
+LA_API la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S,
+                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_stream_t stream);
+LA_API la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t* accepted,
+                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_stream_t stream);
+
+/*
  * Reads the device status word of the current device (synchronizes the
  * device).  *out receives LA_OK or LA_ERR_TIMEOUT; clear != 0 resets it.
  */

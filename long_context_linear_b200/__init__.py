@@ -19,7 +19,8 @@ import torch
 from . import _abi
 from ._abi import LAError, lib
 
-__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "decode_step", "device_status", "LAError",
+__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "decode_step", "decode_verify", "decode_commit",
+           "device_status", "LAError",
            "lib", "prefill_workspace_size", "prefill_varlen_workspace_size"]
 
 _DT = {torch.bfloat16: _abi.LA_BF16, torch.float32: _abi.LA_FP32}
@@ -203,6 +204,49 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tens
                                             _dtype_code(q), _STATE_DT[S.dtype], _stream(q.device)),
                    "la_decode_step_state")
     return out
+
+
+def decode_verify(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Outputs for m draft tokens per (batch, head) without changing S.
+
+    q, k, v: [B, H, m, d] (1 <= m <= 16); S: fp32 [B, H, d, d] (read only).
+    Returns o [B, H, m, d] with o_t = q_t (S + sum_{s<=t} k_s (x) v_s).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, q.device)
+    _need(S, "S", torch.float32, q.device)
+    if q.dim() != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B, H, m, dk] and v [B, H, m, dv]")
+    B, H, m, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(S.shape) != (B, H, dk, dv):
+        raise ValueError("S must be [B, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, H, m, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, q.device)
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, m, dk, dv,
+                                        _dtype_code(q), _stream(q.device)), "la_decode_verify")
+    return out
+
+
+def decode_commit(k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, accepted: torch.Tensor) -> None:
+    """S <- S + sum_{t < accepted[b]} k_t (x) v_t in place (the accepted drafts).
+
+    k, v: [B, H, m, d]; S: fp32 [B, H, d, d]; accepted: int32 [B] on the device.
+    """
+    _need(k, "k", k.dtype, k.device)
+    _need(v, "v", k.dtype, k.device)
+    _need(S, "S", torch.float32, k.device)
+    _need(accepted, "accepted", torch.int32, k.device)
+    B, H, m, dk = k.shape
+    dv = v.shape[-1]
+    if tuple(S.shape) != (B, H, dk, dv) or accepted.numel() != B:
+        raise ValueError("S must be [B, H, dk, dv] and accepted [B]")
+    with torch.cuda.device(k.device):
+        _abi.check(lib.la_decode_commit(_ptr(k), _ptr(v), _ptr(S), _ptr(accepted), B, H, m, dk, dv,
+                                        _dtype_code(k), _stream(k.device)), "la_decode_commit")
 
 
 def device_status(clear: bool = True) -> int:

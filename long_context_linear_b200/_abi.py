@@ -37,12 +37,15 @@ SIGNATURES = {
                                _vp, _sz, _vp]),
     "la_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "la_decode_step_state": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_verify": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_commit": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
     "la_selftest_wait_timeout": (_i, [_i, _vp]),
     "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
 
 NOALLOC_MAX_SEQS = 4096  # LA_NOALLOC_MAX_SEQS in include/la.h
+MAX_DRAFTS = 16  # largest m of la_decode_verify / la_decode_commit
 
 
 class LAError(RuntimeError):

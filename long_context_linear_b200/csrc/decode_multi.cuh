@@ -1,0 +1,130 @@
+// Speculative decoding over m draft tokens per (sequence, head): verify, then commit.
+//
+// A draft model proposes m tokens; the target must give o_t = q_t S_t for all
+// of them, then keep the state of the accepted prefix only.  The state cannot
+// simply be truncated after the fact (page "MiniMax: «Почему M2 …»",
+// section 4, and page "MiniMax-M1で理解する…", the infrastructure list: a
+// recurrent state has no per-token entries to drop), so the two halves are
+// separate:
+//
+//   verify:  o_t = q_t S_0 + sum_{s <= t} (q_t . k_s) v_s      S_0 is only read
+//            (the recurrence S_t = S_0 + sum_{s<=t} k_s v_s^T of page
+//            "MiniMax-M1で理解する…", section "線形アテンションの数学的基礎",
+//            expanded for the m tokens)
+//   commit:  S <- S + sum_{t < a} k_t v_t^T, a = accepted count, in place, one
+//            fused multiply-add per token in token order (so the committed
+//            state is bit-identical to a single decode steps)
+//
+// Both read the d x d fp32 state once (commit also writes it): 3 state passes
+// for m tokens instead of 2 m with m decode steps.  Layout per unit as in
+// decode.cuh: thread = one 16-byte column vector of D/RS rows.
+#pragma once
+#include <cuda_bf16.h>
+#include "decode.cuh"
+
+namespace lcl {
+namespace dmulti {
+
+constexpr int NUM_THREADS = 256;
+constexpr int MAX_M = 16;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(NUM_THREADS)
+verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
+              const float* __restrict__ S, int m) {
+    constexpr int TPR = D / 4;
+    constexpr int RS = NUM_THREADS / TPR;
+    constexpr int RPT = D / RS;
+    __shared__ float qs[MAX_M][D], ks[MAX_M][D], vs[MAX_M][D];
+    __shared__ float A[MAX_M][MAX_M];  // A[t][s] = q_t . k_s, s <= t
+    __shared__ float red[RS][D];
+
+    const long u = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int c4 = tid % TPR, slot = tid / TPR;
+    const float4* Su = reinterpret_cast<const float4*>(S + u * D * D);
+    float4 x[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
+    const long base = u * (long)m * D;
+    for (int e = tid; e < m * D; e += NUM_THREADS) {
+        qs[e / D][e % D] = dec::ld_f(q + base + e);
+        ks[e / D][e % D] = dec::ld_f(k + base + e);
+        vs[e / D][e % D] = dec::ld_f(v + base + e);
+    }
+    __syncthreads();
+    // intra-draft scores
+    for (int p = tid; p < m * m; p += NUM_THREADS) {
+        const int t = p / m, s = p % m;
+        float a = 0.f;
+        if (s <= t) {
+#pragma unroll 8
+            for (int i = 0; i < D; ++i) a = fmaf(qs[t][i], ks[s][i], a);
+        }
+        A[t][s] = a;
+    }
+    // q_t S_0 for every draft token, reduced over row slots
+    for (int t = 0; t < m; ++t) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const float qi = qs[t][slot + r * RS];
+            acc.x = fmaf(qi, x[r].x, acc.x);
+            acc.y = fmaf(qi, x[r].y, acc.y);
+            acc.z = fmaf(qi, x[r].z, acc.z);
+            acc.w = fmaf(qi, x[r].w, acc.w);
+        }
+        *reinterpret_cast<float4*>(&red[slot][4 * c4]) = acc;
+        __syncthreads();
+        if (tid < D) {
+            float sum = 0.f;
+#pragma unroll
+            for (int sl = 0; sl < RS; ++sl) sum += red[sl][tid];
+            for (int s = 0; s <= t; ++s) sum = fmaf(A[t][s], vs[s][tid], sum);
+            dec::st_f(o + base + (long)t * D + tid, sum);
+        }
+        __syncthreads();
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(NUM_THREADS)
+commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restrict__ S,
+              const int* __restrict__ accepted, int H, int m) {
+    constexpr int TPR = D / 4;
+    constexpr int RS = NUM_THREADS / TPR;
+    constexpr int RPT = D / RS;
+    __shared__ float ks[MAX_M][D], vs[MAX_M][D];
+
+    const long u = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int c4 = tid % TPR, slot = tid / TPR;
+    const int a = min(max(accepted[u / H], 0), m);
+    if (a == 0) return;
+    float4* Su = reinterpret_cast<float4*>(S + u * D * D);
+    float4 x[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
+    const long base = u * (long)m * D;
+    for (int e = tid; e < a * D; e += NUM_THREADS) {
+        ks[e / D][e % D] = dec::ld_f(k + base + e);
+        vs[e / D][e % D] = dec::ld_f(v + base + e);
+    }
+    __syncthreads();
+    for (int t = 0; t < a; ++t) {
+        const float4 vj = *reinterpret_cast<const float4*>(&vs[t][4 * c4]);
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const float ki = ks[t][slot + r * RS];
+            x[r].x = fmaf(ki, vj.x, x[r].x);
+            x[r].y = fmaf(ki, vj.y, x[r].y);
+            x[r].z = fmaf(ki, vj.z, x[r].z);
+            x[r].w = fmaf(ki, vj.w, x[r].w);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) __stcs(&Su[(slot + r * RS) * TPR + c4], x[r]);
+}
+
+}  // namespace dmulti
+}  // namespace lcl

@@ -25,6 +25,7 @@
 #include "varlen_order.cuh"
 #include "selftest.cuh"
 #include "seg_prefix.cuh"
+#include "decode_multi.cuh"
 
 namespace lcl {
 
@@ -484,6 +485,72 @@ la_status la_decode_step_state(const void* q, const void* k, const void* v, void
 la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S, int B, int H, int dk,
                          int dv, la_dtype dt, la_stream_t stream) {
     return la_decode_step_state(q, k, v, o, S, B, H, dk, dv, dt, LA_STATE_FP32, stream);
+}
+
+la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S, int B, int H,
+                           int m, int dk, int dv, la_dtype dt, la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
+    if (m < 1 || m > dmulti::MAX_M) return fail(LA_ERR_INVALID_ARG, "m=%d outside 1..%d", m, dmulti::MAX_M);
+    const long U = (long)B * H;
+    if (U == 0) return LA_OK;
+    if (U > (1L << 31) - 1) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (!q || !k || !v || !o || !S) return fail(LA_ERR_INVALID_ARG, "q, k, v, o, S must be non-null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S))
+        return fail(LA_ERR_INVALID_ARG, "all pointers must be 16-byte aligned");
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int grid = (int)U;
+    if (dt == LA_BF16) {
+        using T = __nv_bfloat16;
+        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+    } else {
+        using T = float;
+        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+    }
+    return after_launch("decode_verify launch");
+}
+
+la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t* accepted, int B, int H, int m,
+                           int dk, int dv, la_dtype dt, la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
+    if (m < 1 || m > dmulti::MAX_M) return fail(LA_ERR_INVALID_ARG, "m=%d outside 1..%d", m, dmulti::MAX_M);
+    const long U = (long)B * H;
+    if (U == 0) return LA_OK;
+    if (U > (1L << 31) - 1) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (!k || !v || !S || !accepted) return fail(LA_ERR_INVALID_ARG, "k, v, S, accepted must be non-null");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(S) || (reinterpret_cast<uintptr_t>(accepted) & 3u))
+        return fail(LA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned, accepted 4-byte aligned");
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (env_validate()) {
+        std::vector<int32_t> h(B);
+        cudaError_t e = cudaMemcpyAsync(h.data(), accepted, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "copy accepted for validation");
+        for (int b = 0; b < B; ++b)
+            if (h[b] < 0 || h[b] > m) return fail(LA_ERR_INVALID_ARG, "accepted[%d]=%d outside 0..%d", b, h[b], m);
+    }
+    const int grid = (int)U;
+    if (dt == LA_BF16) {
+        using T = __nv_bfloat16;
+        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+    } else {
+        using T = float;
+        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+    }
+    return after_launch("decode_commit launch");
 }
 
 namespace lcl {

@@ -139,6 +139,34 @@ def test_decode_state_rejects_bad_arguments(lib, kw, status):
     assert _decode_state(lib, **kw) == status
 
 
+def _verify(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, stream=None)
+    a.update(kw)
+    return lib.la_decode_verify(a["q"], a["k"], a["v"], a["o"], a["S"], a["B"], a["H"], a["m"], a["dk"], a["dv"],
+                                a["dt"], a["stream"])
+
+
+def _commit(lib, **kw):
+    a = dict(k=FAKE, v=FAKE, S=FAKE, acc=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, stream=None)
+    a.update(kw)
+    return lib.la_decode_commit(a["k"], a["v"], a["S"], a["acc"], a["B"], a["H"], a["m"], a["dk"], a["dv"], a["dt"],
+                                a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(m=0), 1), (dict(m=17), 1), (dict(S=None), 1), (dict(o=FAKE + 8), 1), (dict(B=-1), 1),
+    (dict(dk=32, dv=32), 2)])
+def test_verify_rejects_bad_arguments(lib, kw, status):
+    assert _verify(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(m=0), 1), (dict(m=17), 1), (dict(acc=None), 1), (dict(acc=FAKE + 2), 1), (dict(S=FAKE + 4), 1),
+    (dict(dk=64, dv=128), 2)])
+def test_commit_rejects_bad_arguments(lib, kw, status):
+    assert _commit(lib, **kw) == status
+
+
 def test_device_status_null(lib):
     assert lib.la_device_status(None, 0) == 1
 
