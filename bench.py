@@ -407,7 +407,7 @@ def run_varlen(args, dist: Dist, pk):
                 frac=gbs / pk["hbm"], tflops_rec=flops_rec(T * H, d) / (ms_step / 1e3) / 1e12, steps=n)
 
 
-def run_prefill8k(args, dist: Dist, pk):
+def run_prefill8k(args, dist: Dist, pk, phi: str = "identity"):
     import long_context_linear_b200 as la
     import synth
     c = PREFILL8K
@@ -418,15 +418,16 @@ def run_prefill8k(args, dist: Dist, pk):
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     n = max(10, min(args.steps, 200))
-    total_ms, per = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s), n, max(3, args.warmup),
-                                   dist, stream)
+    total_ms, per = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, phi=phi), n,
+                                   max(3, args.warmup), dist, stream)
     total_ms = dist.max(total_ms)
     ms_step = total_ms / n
     byts = prefill_bytes(B, H, N, d)
     gbs = byts / (ms_step / 1e3) / 1e9
     del q, k, v, o, s
     torch.cuda.empty_cache()
-    return dict(workload="prefill B=4 H=32 N=8192 d=128 bf16", tokens_per_s=B * N * dist.world / (ms_step / 1e3),
+    return dict(workload=f"prefill B=4 H=32 N=8192 d=128 bf16, feature map {phi}",
+                tokens_per_s=B * N * dist.world / (ms_step / 1e3),
                 ms_per_step=ms_step, hbm_gbs=gbs, frac=gbs / pk["hbm"],
                 tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
                 l2="inputs (1 GiB) larger than L2")
@@ -567,6 +568,7 @@ def main():
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
+        extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
         extras["few_heads"] = run_few_heads(args, dist, pk)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:

@@ -63,8 +63,19 @@ typedef enum {
 
 typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
 
-/* Storage format of a decode state (see la_decode_step_state). */
+/* Storage format of a decode state (see la_decode_step_ex). */
 typedef enum { LA_STATE_FP32 = 0, LA_STATE_BF16 = 1, LA_STATE_FP16 = 2 } la_state_dtype;
+
+/*
+ * Element-wise feature map phi on queries and keys.  Page "MiniMax-M1で理解す
+ * る…", section "線形アテンションの数学的基礎", writes linear attention as
+ * phi(Q) (phi(K)^T V) with a generic phi: S_t = S_{t-1} + phi(k_t) v_t^T,
+ * o_t = phi(q_t) S_t.  LA_PHI_ELU1 is elu(x) + 1 (x + 1 for x > 0, exp(x)
+ * otherwise), LA_PHI_RELU is max(x, 0).  phi is evaluated in fp32; on the bf16
+ * tensor-core prefill path its result is rounded to bf16 before the products.
+ * Every entry point without a phi argument uses the identity.
+ */
+typedef enum { LA_PHI_IDENTITY = 0, LA_PHI_ELU1 = 1, LA_PHI_RELU = 2 } la_phi;
 
 /* Same type as cudaStream_t (an opaque CUDA stream handle). */
 typedef struct CUstream_st* la_stream_t;
@@ -105,6 +116,11 @@ LA_API la_status la_prefill(const void* q, const void* k, const void* v, void* o
                      const float* s0, float* s_out,
                      int B, int H, int N, int dk, int dv, la_dtype dt, int chunk,
                      void* workspace, size_t ws_bytes, la_stream_t stream);
+/* la_prefill with a feature map phi on q and k (see la_phi). */
+LA_API la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o,
+                        const float* s0, float* s_out,
+                        int B, int H, int N, int dk, int dv, la_dtype dt, int chunk, la_phi phi,
+                        void* workspace, size_t ws_bytes, la_stream_t stream);
 
 /*
  * Ragged (packed) prefill with prefix resume.
@@ -128,6 +144,12 @@ LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v, 
                             const float* state_pool, int n_pool, const int32_t* init_idx,
                             float* s_out, int H, int dk, int dv, la_dtype dt, int chunk,
                             void* workspace, size_t ws_bytes, la_stream_t stream);
+/* la_prefill_varlen with a feature map phi on q and k (see la_phi). */
+LA_API la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o,
+                               const int32_t* cu_seqlens, int n_seq, int T,
+                               const float* state_pool, int n_pool, const int32_t* init_idx,
+                               float* s_out, int H, int dk, int dv, la_dtype dt, int chunk, la_phi phi,
+                               void* workspace, size_t ws_bytes, la_stream_t stream);
 
 /*
  * One decode step for B*H independent states (page "MiniMax: «Почему M2 …»",
@@ -139,7 +161,7 @@ LA_API la_status la_decode_step(const void* q, const void* k, const void* v, voi
                          int B, int H, int dk, int dv, la_dtype dt, la_stream_t stream);
 
 /*
- * la_decode_step with the state stored in a chosen format, for the study of
+ * la_decode_step with the state stored in a chosen format and a feature map phi, for the study of
  * low-precision state storage that page "MiniMax: «Почему M2 …»", section 4,
  * and page "ノーフリーランチ：MiniMax M2が高効率アテンション機構を解体",
  * infrastructure section, warn about (the state is rewritten at every token,
@@ -149,10 +171,11 @@ LA_API la_status la_decode_step(const void* q, const void* k, const void* v, voi
  *   multiply-add) and rounded to `sdt` to nearest even; o = q S uses the
  *   stored, rounded state.  LA_STATE_FP32 is exactly la_decode_step.
  *   Low-precision storage needs bf16 q, k, v (LA_ERR_UNSUPPORTED otherwise).
+ *   phi (see la_phi) is applied to q and k as they are loaded.
  */
-LA_API la_status la_decode_step_state(const void* q, const void* k, const void* v, void* o, void* S,
-                                      int B, int H, int dk, int dv, la_dtype dt, la_state_dtype sdt,
-                                      la_stream_t stream);
+LA_API la_status la_decode_step_ex(const void* q, const void* k, const void* v, void* o, void* S,
+                                   int B, int H, int dk, int dv, la_dtype dt, la_state_dtype sdt, la_phi phi,
+                                   la_stream_t stream);
 
 /*
  * Speculative decoding over m draft tokens per sequence (1 <= m <= 16): the
@@ -167,12 +190,15 @@ LA_API la_status la_decode_step_state(const void* q, const void* k, const void* 
  *   every head of sequence b; accepted: int32 device [B], values outside
  *   [0, m] are clamped (checked on the host under LA_VALIDATE=1).  The
  *   committed state is bit-identical to accepted[b] calls of la_decode_step.
- * Each call reads the state once (commit also writes it back).
+ * Each call reads the state once (commit also writes it back).  phi (see
+ * la_phi) is applied to q and k as they are loaded; use the same phi for both.
  */
 LA_API la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S,
-                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_stream_t stream);
+                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_phi phi,
+                                  la_stream_t stream);
 LA_API la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t* accepted,
-                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_stream_t stream);
+                                  int B, int H, int m, int dk, int dv, la_dtype dt, la_phi phi,
+                                  la_stream_t stream);
 
 /*
  * Reads the device status word of the current device (synchronizes the

@@ -24,6 +24,13 @@ __all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "decode_step",
            "lib", "prefill_workspace_size", "prefill_varlen_workspace_size"]
 
 _DT = {torch.bfloat16: _abi.LA_BF16, torch.float32: _abi.LA_FP32}
+PHI = {"identity": _abi.LA_PHI_IDENTITY, "elu1": _abi.LA_PHI_ELU1, "relu": _abi.LA_PHI_RELU}
+
+
+def _phi_code(phi: str) -> int:
+    if phi not in PHI:
+        raise ValueError(f"unknown feature map {phi!r}; one of {sorted(PHI)}")
+    return PHI[phi]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -61,11 +68,12 @@ def prefill_varlen_workspace_size(n_seq: int, T: int, H: int, d: int, dtype: tor
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torch.Tensor] = None, *,
             chunk: int = 0, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
-            return_state: bool = True, workspace: Optional[torch.Tensor] = None
+            return_state: bool = True, workspace: Optional[torch.Tensor] = None, phi: str = "identity"
             ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Dense prefill over q, k, v of shape [B, H, N, d]; returns (O, S_N).
 
-    s0 (fp32 [B, H, d, d]) is the state before the first token (zero if None).
+    s0 (fp32 [B, H, d, d]) is the state before the first token (zero if None);
+    phi ("identity", "elu1", "relu") is the feature map on q and k.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype, q.device)
@@ -90,21 +98,22 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torc
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
-        _abi.check(lib.la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(s0), _ptr(s_out),
-                                  B, H, N, dk, dv, dt, chunk, _ptr(workspace), ws_bytes, _stream(q.device)),
-                   "la_prefill")
+        _abi.check(lib.la_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(s0), _ptr(s_out),
+                                     B, H, N, dk, dv, dt, chunk, _phi_code(phi), _ptr(workspace), ws_bytes,
+                                     _stream(q.device)),
+                   "la_prefill_ex")
     return out, s_out
 
 
 def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                    state_pool: Optional[torch.Tensor] = None, init_idx: Optional[torch.Tensor] = None, *,
                    chunk: int = 0, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
-                   return_state: bool = True, workspace: Optional[torch.Tensor] = None
+                   return_state: bool = True, workspace: Optional[torch.Tensor] = None, phi: str = "identity"
                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Packed ragged prefill: q, k [T, H, d], v [T, H, d], cu_seqlens int32 [n_seq + 1].
 
-    Sequence n starts from state_pool[init_idx[n]] when init_idx[n] >= 0.
-    Returns (O [T, H, d], S [n_seq, H, d, d]).
+    Sequence n starts from state_pool[init_idx[n]] when init_idx[n] >= 0;
+    phi is the feature map on q and k.  Returns (O [T, H, d], S [n_seq, H, d, d]).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype, q.device)
@@ -137,10 +146,10 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
-        _abi.check(lib.la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq, T,
-                                         _ptr(state_pool), n_pool, _ptr(init_idx), _ptr(s_out), H, dk, dv, dt,
-                                         chunk, _ptr(workspace), ws_bytes, _stream(q.device)),
-                   "la_prefill_varlen")
+        _abi.check(lib.la_prefill_varlen_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq, T,
+                                            _ptr(state_pool), n_pool, _ptr(init_idx), _ptr(s_out), H, dk, dv, dt,
+                                            chunk, _phi_code(phi), _ptr(workspace), ws_bytes, _stream(q.device)),
+                   "la_prefill_varlen_ex")
     return out, s_out
 
 
@@ -178,7 +187,7 @@ _STATE_DT = {torch.float32: _abi.LA_STATE_FP32, torch.bfloat16: _abi.LA_STATE_BF
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None, phi: str = "identity") -> torch.Tensor:
     """One token per (batch, head): S <- S + k (x) v in place, returns o = q S.
 
     q, k, v: [B, H, d]; S: [B, H, d, d] in fp32, or in bf16 / fp16 (state
@@ -200,14 +209,14 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tens
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _need(out, "out", q.dtype, q.device)
     with torch.cuda.device(q.device):
-        _abi.check(lib.la_decode_step_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, dk, dv,
-                                            _dtype_code(q), _STATE_DT[S.dtype], _stream(q.device)),
-                   "la_decode_step_state")
+        _abi.check(lib.la_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, dk, dv,
+                                         _dtype_code(q), _STATE_DT[S.dtype], _phi_code(phi), _stream(q.device)),
+                   "la_decode_step_ex")
     return out
 
 
 def decode_verify(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
-                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  out: Optional[torch.Tensor] = None, phi: str = "identity") -> torch.Tensor:
     """Outputs for m draft tokens per (batch, head) without changing S.
 
     q, k, v: [B, H, m, d] (1 <= m <= 16); S: fp32 [B, H, d, d] (read only).
@@ -227,11 +236,12 @@ def decode_verify(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Te
     _need(out, "out", q.dtype, q.device)
     with torch.cuda.device(q.device):
         _abi.check(lib.la_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), B, H, m, dk, dv,
-                                        _dtype_code(q), _stream(q.device)), "la_decode_verify")
+                                        _dtype_code(q), _phi_code(phi), _stream(q.device)), "la_decode_verify")
     return out
 
 
-def decode_commit(k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, accepted: torch.Tensor) -> None:
+def decode_commit(k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, accepted: torch.Tensor, *,
+                  phi: str = "identity") -> None:
     """S <- S + sum_{t < accepted[b]} k_t (x) v_t in place (the accepted drafts).
 
     k, v: [B, H, m, d]; S: fp32 [B, H, d, d]; accepted: int32 [B] on the device.
@@ -246,7 +256,7 @@ def decode_commit(k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, accepted: t
         raise ValueError("S must be [B, H, dk, dv] and accepted [B]")
     with torch.cuda.device(k.device):
         _abi.check(lib.la_decode_commit(_ptr(k), _ptr(v), _ptr(S), _ptr(accepted), B, H, m, dk, dv,
-                                        _dtype_code(k), _stream(k.device)), "la_decode_commit")
+                                        _dtype_code(k), _phi_code(phi), _stream(k.device)), "la_decode_commit")
 
 
 def device_status(clear: bool = True) -> int:

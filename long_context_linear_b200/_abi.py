@@ -21,6 +21,9 @@ LA_FP32 = 1
 LA_STATE_FP32 = 0
 LA_STATE_BF16 = 1
 LA_STATE_FP16 = 2
+LA_PHI_IDENTITY = 0
+LA_PHI_ELU1 = 1
+LA_PHI_RELU = 2
 
 # name -> (restype, argtypes), mirroring include/la.h
 _vp = ctypes.c_void_p
@@ -32,13 +35,16 @@ SIGNATURES = {
     "la_version": (_i, []),
     "la_prefill_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "la_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "la_prefill_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "la_prefill_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "la_prefill_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i,
                                _vp, _sz, _vp]),
+    "la_prefill_varlen_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                  _vp, _sz, _vp]),
     "la_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
-    "la_decode_step_state": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
-    "la_decode_verify": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
-    "la_decode_commit": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_step_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_verify": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_decode_commit": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
     "la_selftest_wait_timeout": (_i, [_i, _vp]),
     "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),

@@ -13,10 +13,12 @@
 // storage the same section warns about).  The update is always computed in
 // fp32: S_new = RN_fp32(S_stored + k_i v_j) (one fused multiply-add, the
 // product of two bf16 inputs being exact in fp32), then rounded to the storage
-// format to nearest even; o uses the stored (rounded) state.
+// format to nearest even; o uses the stored (rounded) state.  A feature map
+// phi (phi.cuh) is applied to q and k as they are loaded.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include "phi.cuh"
 
 namespace lcl {
 namespace dec {
@@ -89,7 +91,7 @@ template <> struct Vec<__half> {
 template <typename T, typename SS, int D>
 __global__ void __launch_bounds__(NUM_THREADS)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
-                   SS* __restrict__ S) {
+                   SS* __restrict__ S, int phi) {
     constexpr int E = Vec<SS>::E;          // state values per 16-byte vector
     constexpr int TPR = D / E;             // threads per row
     constexpr int RS = NUM_THREADS / TPR;  // row slots
@@ -107,8 +109,8 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 #pragma unroll
     for (int m = 0; m < RPT; ++m) x[m] = __ldcs(&Su[(slot + m * RS) * TPR + cv]);
     if (tid < D) {
-        qs[tid] = ld_f(q + u * D + tid);
-        ks[tid] = ld_f(k + u * D + tid);
+        qs[tid] = apply_phi(ld_f(q + u * D + tid), phi);
+        ks[tid] = apply_phi(ld_f(k + u * D + tid), phi);
         vs[tid] = ld_f(v + u * D + tid);
     }
     __syncthreads();

@@ -15,6 +15,7 @@
 //            fused multiply-add per token in token order (so the committed
 //            state is bit-identical to a single decode steps)
 //
+// A feature map phi (phi.cuh) is applied to q and k as they are loaded.
 // Both read the d x d fp32 state once (commit also writes it): 3 state passes
 // for m tokens instead of 2 m with m decode steps.  Layout per unit as in
 // decode.cuh: thread = one 16-byte column vector of D/RS rows.
@@ -31,7 +32,7 @@ constexpr int MAX_M = 16;
 template <typename T, int D>
 __global__ void __launch_bounds__(NUM_THREADS)
 verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
-              const float* __restrict__ S, int m) {
+              const float* __restrict__ S, int m, int phi) {
     constexpr int TPR = D / 4;
     constexpr int RS = NUM_THREADS / TPR;
     constexpr int RPT = D / RS;
@@ -48,8 +49,8 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
     const long base = u * (long)m * D;
     for (int e = tid; e < m * D; e += NUM_THREADS) {
-        qs[e / D][e % D] = dec::ld_f(q + base + e);
-        ks[e / D][e % D] = dec::ld_f(k + base + e);
+        qs[e / D][e % D] = apply_phi(dec::ld_f(q + base + e), phi);
+        ks[e / D][e % D] = apply_phi(dec::ld_f(k + base + e), phi);
         vs[e / D][e % D] = dec::ld_f(v + base + e);
     }
     __syncthreads();
@@ -90,7 +91,7 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 template <typename T, int D>
 __global__ void __launch_bounds__(NUM_THREADS)
 commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restrict__ S,
-              const int* __restrict__ accepted, int H, int m) {
+              const int* __restrict__ accepted, int H, int m, int phi) {
     constexpr int TPR = D / 4;
     constexpr int RS = NUM_THREADS / TPR;
     constexpr int RPT = D / RS;
@@ -107,7 +108,7 @@ commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restric
     for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
     const long base = u * (long)m * D;
     for (int e = tid; e < a * D; e += NUM_THREADS) {
-        ks[e / D][e % D] = dec::ld_f(k + base + e);
+        ks[e / D][e % D] = apply_phi(dec::ld_f(k + base + e), phi);
         vs[e / D][e % D] = dec::ld_f(v + base + e);
     }
     __syncthreads();

@@ -146,6 +146,12 @@ bool env_validate() {
     return v && v[0] == '1';
 }
 
+la_status check_phi(la_phi phi) {
+    if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1 && phi != LA_PHI_RELU)
+        return fail(LA_ERR_INVALID_ARG, "unknown feature map %d", (int)phi);
+    return LA_OK;
+}
+
 la_status check_dims(int dk, int dv, la_dtype dt) {
     if (dt != LA_BF16 && dt != LA_FP32) return fail(LA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     if (dk <= 0 || dv <= 0) return fail(LA_ERR_INVALID_ARG, "dk=%d dv=%d must be positive", dk, dv);
@@ -199,13 +205,14 @@ la_status launch_simt(int d, int chunk, int grid, const void* q, const void* k, 
 namespace lcl {
 namespace {
 template <typename T, typename SS>
-void launch_decode(int dk, int grid, const void* q, const void* k, const void* v, void* o, void* S, cudaStream_t st) {
+void launch_decode(int dk, int grid, const void* q, const void* k, const void* v, void* o, void* S, int phi,
+                   cudaStream_t st) {
     if (dk == 128)
         dec::decode_step_kernel<T, SS, 128><<<grid, dec::NUM_THREADS, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S);
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S, phi);
     else
         dec::decode_step_kernel<T, SS, 64><<<grid, dec::NUM_THREADS, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S);
+            (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S, phi);
 }
 }  // namespace
 }  // namespace lcl
@@ -274,9 +281,17 @@ size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype d
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
                      int H, int N, int dk, int dv, la_dtype dt, int chunk, void* workspace, size_t ws_bytes,
                      la_stream_t stream) {
+    return la_prefill_ex(q, k, v, o, s0, s_out, B, H, N, dk, dv, dt, chunk, LA_PHI_IDENTITY, workspace, ws_bytes,
+                         stream);
+}
+
+la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
+                        int H, int N, int dk, int dv, la_dtype dt, int chunk, la_phi phi, void* workspace,
+                        size_t ws_bytes, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if ((s = check_phi(phi)) != LA_OK) return s;
     if (B < 0 || H < 0 || N < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d N=%d", B, H, N);
     const long U = (long)B * H;
     if (U > (1L << 30) || (long)N * U > (1L << 40)) return fail(LA_ERR_INVALID_ARG, "problem too large");
@@ -292,7 +307,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
 
     if (!tcpath) {
         simt::Params sp{};
-        sp.mode = 0; sp.N = N; sp.s0 = s0; sp.s_out = s_out;
+        sp.mode = 0; sp.N = N; sp.s0 = s0; sp.s_out = s_out; sp.phi = phi;
         if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)U, q, k, v, o, sp, st);
         return launch_simt<__nv_bfloat16>(dk, chunk, (int)U, q, k, v, o, sp, st);
     }
@@ -308,6 +323,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.status = di->status;
     p.n_seg = 1;
+    p.phi = phi;
     if (N == 0 && !s_out) return LA_OK;
     int seg_len;
     int P = plan_segments(U, N, di->sms, &seg_len);
@@ -369,9 +385,18 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
                             int n_seq, int T, const float* state_pool, int n_pool, const int32_t* init_idx,
                             float* s_out, int H, int dk, int dv, la_dtype dt, int chunk, void* workspace,
                             size_t ws_bytes, la_stream_t stream) {
+    return la_prefill_varlen_ex(q, k, v, o, cu_seqlens, n_seq, T, state_pool, n_pool, init_idx, s_out, H, dk, dv, dt,
+                                chunk, LA_PHI_IDENTITY, workspace, ws_bytes, stream);
+}
+
+la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                               int n_seq, int T, const float* state_pool, int n_pool, const int32_t* init_idx,
+                               float* s_out, int H, int dk, int dv, la_dtype dt, int chunk, la_phi phi,
+                               void* workspace, size_t ws_bytes, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if ((s = check_phi(phi)) != LA_OK) return s;
     if (n_seq < 0 || T < 0 || H < 0 || n_pool < 0)
         return fail(LA_ERR_INVALID_ARG, "negative size n_seq=%d T=%d H=%d n_pool=%d", n_seq, T, H, n_pool);
     if (n_seq == 0 || H == 0) return LA_OK;
@@ -414,7 +439,7 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
     if (!tcpath) {
         simt::Params sp{};
         sp.mode = 1; sp.H = H; sp.cu_seqlens = cu_seqlens; sp.pool = state_pool; sp.init_idx = init_idx;
-        sp.s_out = s_out;
+        sp.s_out = s_out; sp.phi = phi;
         const long grid = (long)n_seq * H;
         if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)grid, q, k, v, o, sp, st);
         return launch_simt<__nv_bfloat16>(dk, chunk, (int)grid, q, k, v, o, sp, st);
@@ -427,6 +452,7 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
     tc::Params p{};
     p.mode = 1;
     p.n_seg = 1;
+    p.phi = phi;
     p.n_items = (int)((long)n_seq * H * tc::NVS);
     p.H = H;
     p.dv = dv;
@@ -450,11 +476,12 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o
     return after_launch("prefill_tc (varlen) launch");
 }
 
-la_status la_decode_step_state(const void* q, const void* k, const void* v, void* o, void* S, int B, int H, int dk,
-                               int dv, la_dtype dt, la_state_dtype sdt, la_stream_t stream) {
+la_status la_decode_step_ex(const void* q, const void* k, const void* v, void* o, void* S, int B, int H, int dk,
+                            int dv, la_dtype dt, la_state_dtype sdt, la_phi phi, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if ((s = check_phi(phi)) != LA_OK) return s;
     if (sdt != LA_STATE_FP32 && sdt != LA_STATE_BF16 && sdt != LA_STATE_FP16)
         return fail(LA_ERR_INVALID_ARG, "unknown state dtype %d", (int)sdt);
     if (sdt != LA_STATE_FP32 && dt != LA_BF16)
@@ -471,27 +498,28 @@ la_status la_decode_step_state(const void* q, const void* k, const void* v, void
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int grid = (int)U;
     if (dt == LA_FP32) {
-        launch_decode<float, float>(dk, grid, q, k, v, o, S, st);
+        launch_decode<float, float>(dk, grid, q, k, v, o, S, phi, st);
     } else if (sdt == LA_STATE_FP32) {
-        launch_decode<__nv_bfloat16, float>(dk, grid, q, k, v, o, S, st);
+        launch_decode<__nv_bfloat16, float>(dk, grid, q, k, v, o, S, phi, st);
     } else if (sdt == LA_STATE_BF16) {
-        launch_decode<__nv_bfloat16, __nv_bfloat16>(dk, grid, q, k, v, o, S, st);
+        launch_decode<__nv_bfloat16, __nv_bfloat16>(dk, grid, q, k, v, o, S, phi, st);
     } else {
-        launch_decode<__nv_bfloat16, __half>(dk, grid, q, k, v, o, S, st);
+        launch_decode<__nv_bfloat16, __half>(dk, grid, q, k, v, o, S, phi, st);
     }
     return after_launch("decode_step launch");
 }
 
 la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* S, int B, int H, int dk,
                          int dv, la_dtype dt, la_stream_t stream) {
-    return la_decode_step_state(q, k, v, o, S, B, H, dk, dv, dt, LA_STATE_FP32, stream);
+    return la_decode_step_ex(q, k, v, o, S, B, H, dk, dv, dt, LA_STATE_FP32, LA_PHI_IDENTITY, stream);
 }
 
 la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S, int B, int H,
-                           int m, int dk, int dv, la_dtype dt, la_stream_t stream) {
+                           int m, int dk, int dv, la_dtype dt, la_phi phi, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if ((s = check_phi(phi)) != LA_OK) return s;
     if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
     if (m < 1 || m > dmulti::MAX_M) return fail(LA_ERR_INVALID_ARG, "m=%d outside 1..%d", m, dmulti::MAX_M);
     const long U = (long)B * H;
@@ -506,21 +534,22 @@ la_status la_decode_verify(const void* q, const void* k, const void* v, void* o,
     const int grid = (int)U;
     if (dt == LA_BF16) {
         using T = __nv_bfloat16;
-        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
-        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
+        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
     } else {
         using T = float;
-        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
-        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m);
+        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
+        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
     }
     return after_launch("decode_verify launch");
 }
 
 la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t* accepted, int B, int H, int m,
-                           int dk, int dv, la_dtype dt, la_stream_t stream) {
+                           int dk, int dv, la_dtype dt, la_phi phi, la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
+    if ((s = check_phi(phi)) != LA_OK) return s;
     if (B < 0 || H < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d", B, H);
     if (m < 1 || m > dmulti::MAX_M) return fail(LA_ERR_INVALID_ARG, "m=%d outside 1..%d", m, dmulti::MAX_M);
     const long U = (long)B * H;
@@ -543,12 +572,12 @@ la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t
     const int grid = (int)U;
     if (dt == LA_BF16) {
         using T = __nv_bfloat16;
-        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
-        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
+        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
     } else {
         using T = float;
-        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
-        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m);
+        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
+        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
     }
     return after_launch("decode_commit launch");
 }

@@ -11,6 +11,7 @@
 // One CTA per (unit | sequence, head); the whole d x d fp32 state lives in
 // shared memory.  The chunk length CS (32 or 64) is a template parameter.
 #pragma once
+#include "phi.cuh"
 #include <cuda_bf16.h>
 
 namespace lcl {
@@ -27,6 +28,7 @@ struct Params {
     const float* pool;      // packed: [n_pool][H][d][d] or null
     const int* init_idx;    // packed: [n_seq] or null
     float* s_out;           // [U | n_seq*H][d][d] or null
+    int phi;                // feature map applied to q and k (phi.cuh)
 };
 
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -83,8 +85,8 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             float a = 0.f, b = 0.f, cc = 0.f;
             if (t < rows) {
                 const long g = (row0 + (long)(c0 + t) * row_stride) * D + i;
-                a = to_f(q[g]);
-                b = to_f(k[g]);
+                a = apply_phi(to_f(q[g]), p.phi);
+                b = apply_phi(to_f(k[g]), p.phi);
                 cc = to_f(v[g]);
             }
             Qs[t * LD + i] = a;

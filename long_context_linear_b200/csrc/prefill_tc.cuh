@@ -32,6 +32,7 @@
 // the CTA cleanly.
 #pragma once
 #include "sm100.cuh"
+#include "phi.cuh"
 
 namespace lcl {
 namespace tc {
@@ -69,10 +70,11 @@ constexpr int BAR_O_FULL = BAR_P_READY + 2;         // [2]
 constexpr int BAR_O_EMPTY = BAR_O_FULL + 2;         // [2]
 constexpr int BAR_DS_FULL = BAR_O_EMPTY + 2;        // [2]
 constexpr int BAR_DS_EMPTY = BAR_DS_FULL + 2;       // [2]
-constexpr int BAR_DRAIN_A = BAR_DS_EMPTY + 2;
+constexpr int BAR_KPHI_FULL = BAR_DS_EMPTY + 2;     // [K_SLOTS] state (phi applied to K) -> B
+constexpr int BAR_DRAIN_A = BAR_KPHI_FULL + K_SLOTS;
 constexpr int BAR_DRAIN_B = BAR_DRAIN_A + 1;
 constexpr int BAR_COUNT = BAR_DRAIN_B + 1;
-constexpr int BAR_BYTES = 256;
+constexpr int BAR_BYTES = 512;
 static_assert((BAR_COUNT + 2) * 8 <= BAR_BYTES, "barrier area too small");
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB per-block shared memory limit");
@@ -110,6 +112,7 @@ struct Params {
     const float* seg_init; // [U][n_seg][DK][dv]: state before each segment, or null (then s0)
     int s_out_per_seg;     // 1: s_out holds the state after every segment, [U][n_seg][DK][dv]
     int state_only;        // 1: only the state is computed (no Q, no outputs)
+    int phi;               // feature map on q and k (phi.cuh); applied to the tiles in smem
 };
 
 struct Item {
@@ -183,6 +186,31 @@ __device__ __noinline__ void clear_tail_rows(uint8_t* tile, int rows, int ksteps
     fence_proxy_async_smem();
 }
 
+// phi in place on 16-byte vectors [e0, e1) of a tile region, by the 128
+// state-warp threads (t = 0 .. 127); shared-memory addresses.  vec(e) maps a
+// vector index to its address.  Four vectors are loaded before any is
+// transformed.  Out of line: the identity path never runs it and should not
+// carry its code.
+__device__ __noinline__ void phi_region(uint32_t base, uint32_t panel_stride, int per_panel, int n, int t, int phi) {
+#pragma unroll 1
+    for (int e0 = t; e0 < n; e0 += 4 * 128) {
+        uint32_t a[4];
+        uint4 r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + j * 128;
+            a[j] = base + static_cast<uint32_t>(e / per_panel) * panel_stride + static_cast<uint32_t>(e % per_panel) * 16u;
+            if (e < n) r[j] = ld_shared_v4(a[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 y = apply_phi_bf16x8(r[j], phi);
+            if (e0 + j * 128 < n) st_shared_v4(a[j], y.x, y.y, y.z, y.w);
+        }
+    }
+    fence_proxy_async_smem();
+}
+
 // Shared-memory descriptor of K-step kk (16 along the contraction dim):
 // K-major tiles step 32 B inside a 64-column panel (panels `panel` bytes
 // apart), MN-major tiles step 16 rows of 128 B.
@@ -225,6 +253,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     uint64_t* o_empty = bars + BAR_O_EMPTY;    // [2] output -> state
     uint64_t* ds_full = bars + BAR_DS_FULL;    // [2] B -> state
     uint64_t* ds_empty = bars + BAR_DS_EMPTY;  // [2] state -> B
+    uint64_t* kphi_full = bars + BAR_KPHI_FULL;  // [K_SLOTS] state (phi(K) written) -> B, when phi is not the identity
     uint64_t* drain_a = bars + BAR_DRAIN_A;
     uint64_t* drain_b = bars + BAR_DRAIN_B;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + BAR_COUNT);
@@ -241,6 +270,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             mbar_init(&q_empty[i], 1);
         }
         for (int i = 0; i < K_SLOTS; ++i) {
+            mbar_init(&kphi_full[i], 4);
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], p.state_only ? 1 : 2);
             mbar_init(&s_full[i], 4);
@@ -431,7 +461,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     const int rows = len - c0;
                     const int ksteps = (p.mode == 1 && rows < C) ? (rows + 15) >> 4 : C / 16;
                     // dS = K^T V   (A: K MN-major over 2 panels, B: V MN-major)
-                    if (!mbar_wait(&k_full[ks], (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                    uint64_t* kready = p.phi != PHI_IDENTITY ? &kphi_full[ks] : &k_full[ks];
+                    if (!mbar_wait(kready, (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                     if (!mbar_wait(&v_full[vc], (g / V_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                     if (ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
                     if (g >= 2 && !mbar_wait(&ds_empty[b], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
@@ -543,7 +574,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     // the [P|O] product of this chunk also needs Q_c, K_c and the O
                     // buffer it writes (last used by chunk c - 2) drained
                     if (!warp_wait(&q_full[g % Q_SLOTS], (g / Q_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                }
+                if (p.phi != PHI_IDENTITY || !p.state_only) {
                     if (!warp_wait(&k_full[ks], (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
+                }
+                if (p.phi != PHI_IDENTITY) {
+                    // phi(K_c), then phi(Q_c), in place, before the tensor cores read
+                    // them (the S^T rows behind K are left alone); K first, so that
+                    // K^T V can start while Q is mapped
+                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, 2 * PANEL / 16, i, p.phi);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&kphi_full[ks]);
+                    if (!p.state_only)
+                        phi_region(smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q), PANEL, PANEL / 16, 2 * PANEL / 16, i,
+                                   p.phi);
+                }
+                if (!p.state_only) {
                     if (g >= 2 && !warp_wait(&o_empty[g & 1], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
                     tc_fence_before();

@@ -255,6 +255,13 @@ __device__ __forceinline__ void st_shared_b32(uint32_t saddr, uint32_t a) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(a) : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(saddr)
+                 : "memory");
+    return r;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");

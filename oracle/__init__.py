@@ -16,6 +16,10 @@ What it computes (page "MiniMax-M1ã§ç†è§£ã™ã‚‹ï¼šå¤§è¦æ¨¡è¨€èªãƒ¢ãƒ‡ãƒ«ã®ã
 * one decode step  S <- S + k v^T, o = q S                          (``decode``)
 * packed ragged batches with an optional resumed state per sequence (``varlen``).
 
+Every function takes ``phi`` (None / "identity", "elu1", "relu"): the
+element-wise feature map of the same page's phi(Q)(phi(K)^T V), applied in
+float64 to q and k before the recurrence (``feature_map``).
+
 Inputs are the exact stored values (bf16 or fp32) widened to float64; all
 arithmetic is float64.  Pins: ``tests/test_oracle.py``.  No function here is
 "parity unpinned".
@@ -90,8 +94,20 @@ def _ptr(a: Optional[np.ndarray]):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def _dense(fn, q, k, v, s0):
-    q, k, v, s0 = _f64(q), _f64(k), _f64(v), _f64(s0)
+def feature_map(x, phi: Optional[str]) -> np.ndarray:
+    """phi applied element-wise in float64: identity, elu(x) + 1 or relu(x)."""
+    x = _f64(x)
+    if phi in (None, "identity"):
+        return x
+    if phi == "elu1":
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    if phi == "relu":
+        return np.maximum(x, 0.0)
+    raise ValueError(f"unknown feature map {phi!r}")
+
+
+def _dense(fn, q, k, v, s0, phi=None):
+    q, k, v, s0 = feature_map(q, phi), feature_map(k, phi), _f64(v), _f64(s0)
     *lead, N, dk = q.shape
     dv = v.shape[-1]
     assert k.shape == q.shape and tuple(v.shape[:-1]) == tuple(q.shape[:-1])
@@ -104,19 +120,19 @@ def _dense(fn, q, k, v, s0):
     return o, s_out
 
 
-def recurrent(q, k, v, s0=None) -> Tuple[np.ndarray, np.ndarray]:
+def recurrent(q, k, v, s0=None, phi=None) -> Tuple[np.ndarray, np.ndarray]:
     """Token-by-token recurrence on dense [..., N, d] inputs -> (O, S_N)."""
-    return _dense(_load().oracle_recurrent, q, k, v, s0)
+    return _dense(_load().oracle_recurrent, q, k, v, s0, phi)
 
 
-def quadratic(q, k, v, s0=None) -> Tuple[np.ndarray, np.ndarray]:
+def quadratic(q, k, v, s0=None, phi=None) -> Tuple[np.ndarray, np.ndarray]:
     """Masked quadratic form (Q K^T âŠ™ M) V + Q S0 and S0 + K^T V (small N)."""
-    return _dense(_load().oracle_quadratic, q, k, v, s0)
+    return _dense(_load().oracle_quadratic, q, k, v, s0, phi)
 
 
-def decode(q, k, v, S) -> Tuple[np.ndarray, np.ndarray]:
+def decode(q, k, v, S, phi=None) -> Tuple[np.ndarray, np.ndarray]:
     """One decode step: returns (o, S_new); the input S is not modified."""
-    q, k, v = _f64(q), _f64(k), _f64(v)
+    q, k, v = feature_map(q, phi), feature_map(k, phi), _f64(v)
     S = _f64(S).copy()
     dk, dv = q.shape[-1], v.shape[-1]
     U = int(np.prod(q.shape[:-1]))
@@ -125,9 +141,9 @@ def decode(q, k, v, S) -> Tuple[np.ndarray, np.ndarray]:
     return o, S
 
 
-def varlen(q, k, v, cu_seqlens, state_pool=None, init_idx=None):
+def varlen(q, k, v, cu_seqlens, state_pool=None, init_idx=None, phi=None):
     """Packed ragged batch: q,k [T,H,dk], v [T,H,dv] -> (O [T,H,dv], S [n_seq,H,dk,dv])."""
-    q, k, v = _f64(q), _f64(k), _f64(v)
+    q, k, v = feature_map(q, phi), feature_map(k, phi), _f64(v)
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     T, H, dk = q.shape
     dv = v.shape[-1]

@@ -124,38 +124,39 @@ def test_decode_rejects_bad_arguments(lib, kw, status):
 
 
 def _decode_state(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, dk=128, dv=128, dt=0, sdt=1, stream=None)
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, dk=128, dv=128, dt=0, sdt=1, phi=0, stream=None)
     a.update(kw)
-    return lib.la_decode_step_state(a["q"], a["k"], a["v"], a["o"], a["S"], a["B"], a["H"], a["dk"], a["dv"],
-                                    a["dt"], a["sdt"], a["stream"])
+    return lib.la_decode_step_ex(a["q"], a["k"], a["v"], a["o"], a["S"], a["B"], a["H"], a["dk"], a["dv"],
+                                 a["dt"], a["sdt"], a["phi"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,status", [
     (dict(sdt=3), 1), (dict(sdt=-1), 1),   # unknown storage format
     (dict(dt=1, sdt=1), 2),                # a bf16 state needs bf16 inputs
     (dict(dt=1, sdt=2), 2),                # ... as does an fp16 state
-    (dict(S=None), 1), (dict(S=FAKE + 8), 1), (dict(B=-1), 1), (dict(dk=64, dv=128), 2)])
+    (dict(S=None), 1), (dict(S=FAKE + 8), 1), (dict(B=-1), 1), (dict(dk=64, dv=128), 2),
+    (dict(phi=3), 1), (dict(phi=-1), 1)])
 def test_decode_state_rejects_bad_arguments(lib, kw, status):
     assert _decode_state(lib, **kw) == status
 
 
 def _verify(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, stream=None)
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, phi=0, stream=None)
     a.update(kw)
     return lib.la_decode_verify(a["q"], a["k"], a["v"], a["o"], a["S"], a["B"], a["H"], a["m"], a["dk"], a["dv"],
-                                a["dt"], a["stream"])
+                                a["dt"], a["phi"], a["stream"])
 
 
 def _commit(lib, **kw):
-    a = dict(k=FAKE, v=FAKE, S=FAKE, acc=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, stream=None)
+    a = dict(k=FAKE, v=FAKE, S=FAKE, acc=FAKE, B=2, H=2, m=4, dk=128, dv=128, dt=0, phi=0, stream=None)
     a.update(kw)
     return lib.la_decode_commit(a["k"], a["v"], a["S"], a["acc"], a["B"], a["H"], a["m"], a["dk"], a["dv"], a["dt"],
-                                a["stream"])
+                                a["phi"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,status", [
     (dict(m=0), 1), (dict(m=17), 1), (dict(S=None), 1), (dict(o=FAKE + 8), 1), (dict(B=-1), 1),
-    (dict(dk=32, dv=32), 2)])
+    (dict(dk=32, dv=32), 2), (dict(phi=7), 1)])
 def test_verify_rejects_bad_arguments(lib, kw, status):
     assert _verify(lib, **kw) == status
 
@@ -165,6 +166,11 @@ def test_verify_rejects_bad_arguments(lib, kw, status):
     (dict(dk=64, dv=128), 2)])
 def test_commit_rejects_bad_arguments(lib, kw, status):
     assert _commit(lib, **kw) == status
+
+
+def test_prefill_ex_rejects_unknown_feature_map(lib):
+    st = lib.la_prefill_ex(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 128, 128, 0, 0, 5, None, 0, None)
+    assert st == 1
 
 
 def test_device_status_null(lib):

@@ -1,0 +1,124 @@
+"""Feature maps phi (identity, elu + 1, relu) on every path, against the fp64
+oracle with the same phi applied in float64 (page "MiniMax-M1で理解する…",
+section "線形アテンションの数学的基礎": phi(Q) (phi(K)^T V))."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.parity import assert_out, assert_state
+
+pytestmark = pytest.mark.gpu
+
+PHIS = ["elu1", "relu"]
+# On the bf16 tensor-core prefill phi(q), phi(k) are tensor-core operands, so
+# they are rounded to bf16: relu(x) of a bf16 x is exact, elu(x) + 1 is not,
+# and the state then inherits that operand rounding (up to 2^-9 relative per
+# element of phi(k)); its bar there is the output's 5e-3.  The fp32 paths keep
+# phi in fp32 and meet the 1e-4 state bar.
+TC_STATE_TOL = {"elu1": 5e-3, "relu": 1e-4}
+
+
+@pytest.fixture(scope="module")
+def la():
+    import long_context_linear_b200 as la
+    return la
+
+
+def _state(U, d, seed):
+    return synth.outer_product_state(U, d, d, [400] * U, seed=seed)
+
+
+@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("B,H,N", [(1, 2, 1), (1, 2, 200), (2, 3, 1000), (1, 1, 4096 + 33)])
+def test_tc_prefill_with_phi(la, oracle_mod, phi, B, H, N):
+    q, k, v = synth.dense(B, H, N, 128, "bf16", seed=N + 3)
+    s0 = _state(B * H, 128, seed=N).view(B, H, 128, 128)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), s0.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, s0, phi=phi)
+    assert_out(o.cpu(), ro, torch.bfloat16, 2)
+    assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_tc_prefill_with_phi_and_segments(la, oracle_mod, monkeypatch, phi):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", "3")
+    q, k, v = synth.dense(1, 2, 3000, 128, "bf16", seed=77)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, phi=phi)
+    assert_out(o.cpu(), ro, torch.bfloat16, 2)
+    assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])
+
+
+@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("dtype,d", [("fp32", 64), ("bf16", 64), ("fp32", 128)])
+def test_ffma_prefill_with_phi(la, oracle_mod, phi, dtype, d):
+    q, k, v = synth.dense(2, 2, 300, d, dtype, seed=d + 1)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, phi=phi)
+    assert_out(o.cpu(), ro, q.dtype, 2)
+    assert_state(s.cpu(), rs, 2)
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_varlen_with_phi(la, oracle_mod, phi):
+    lens = [0, 1, 130, 257, 1000]
+    cu = synth.cu_seqlens(lens)
+    T, H, d = int(cu[-1]), 2, 128
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=5)
+    pool = _state(2 * H, d, seed=6).view(2, H, d, d)
+    init = torch.tensor([-1, 0, 1, -1, 0], dtype=torch.int32)
+    o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), pool.cuda(), init.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, init, phi=phi)
+    assert_out(o.cpu()[None], ro[None], torch.bfloat16, 1)
+    assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_decode_with_phi(la, oracle_mod, phi):
+    B, H, d, T = 2, 3, 128, 8
+    S = _state(B * H, d, seed=8).view(B, H, d, d)
+    Sd = S.cuda()
+    S_ref = S.double().numpy()
+    qs, ks, vs = synth.qkv((T, B, H, d), d, "bf16", seed=9)
+    for t in range(T):
+        o = la.decode_step(qs[t].cuda(), ks[t].cuda(), vs[t].cuda(), Sd, phi=phi)
+        ro, S_ref = oracle_mod.decode(qs[t], ks[t], vs[t], S_ref, phi=phi)
+        assert_out(o.cpu(), ro, torch.bfloat16, 2)
+    assert_state(Sd.cpu(), S_ref, 2, tol=1e-6)
+    assert la.device_status() == 0
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_verify_and_commit_with_phi(la, oracle_mod, phi):
+    B, H, m, d = 2, 2, 5, 128
+    S = _state(B * H, d, seed=10).view(B, H, d, d)
+    q, k, v = synth.qkv((B, H, m, d), d, "bf16", seed=11)
+    Sd = S.cuda()
+    o = la.decode_verify(q.cuda(), k.cuda(), v.cuda(), Sd, phi=phi)
+    ro, rs = oracle_mod.recurrent(q, k, v, S, phi=phi)
+    assert_out(o.cpu(), ro, torch.bfloat16, 2)
+    la.decode_commit(k.cuda(), v.cuda(), Sd, torch.full((B,), m, dtype=torch.int32, device="cuda"), phi=phi)
+    assert_state(Sd.cpu(), rs, 2, tol=1e-6)
+    assert la.device_status() == 0
+
+
+def test_identity_phi_is_the_default(la):
+    q, k, v = (x.cuda() for x in synth.dense(1, 2, 700, 128, "bf16", seed=12))
+    o1, s1 = la.prefill(q, k, v)
+    o2, s2 = la.prefill(q, k, v, phi="identity")
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_unknown_phi_is_rejected(la):
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        la.prefill(q, q, q, phi="tanh")

@@ -342,3 +342,26 @@ def test_lowp_decode_fp32_tracks_the_fp64_recurrence(oracle_mod):
         o, S = lowp.decode_lowp(q[t], k[t], v[t], S, "fp32")
     assert _rel(S.astype(np.float64), S64) < 1e-6
     assert _rel(o, o_ref) < 1e-6
+
+
+# ------------------------------------------------------------- feature maps
+
+def test_feature_maps_closed_forms(oracle_mod):
+    x = np.array([-2.0, -1.0, 0.0, 0.5, 3.0])
+    np.testing.assert_array_equal(oracle_mod.feature_map(x, None), x)
+    np.testing.assert_allclose(oracle_mod.feature_map(x, "elu1"), [np.exp(-2.0), np.exp(-1.0), 1.0, 1.5, 4.0],
+                               rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(oracle_mod.feature_map(x, "relu"), [0.0, 0.0, 0.0, 0.5, 3.0])
+
+
+@pytest.mark.parametrize("phi", ["elu1", "relu"])
+def test_feature_map_enters_only_through_q_and_k(oracle_mod, phi):
+    """With phi the recurrence is the identity-phi recurrence on phi(q), phi(k);
+    brute force of o_t = sum_{s<=t} (phi(q_t).phi(k_s)) v_s + phi(q_t) S0."""
+    q, k, v, s0 = _rand((7, 5), 41), _rand((7, 5), 42), _rand((7, 4), 43), _rand((5, 4), 44)
+    o, S = oracle_mod.recurrent(q, k, v, s0, phi=phi)
+    fq, fk = oracle_mod.feature_map(q, phi), oracle_mod.feature_map(k, phi)
+    ob, Sb = _brute(fq, fk, v, s0)
+    assert _rel(o, ob) < 1e-12 and _rel(S, Sb) < 1e-12
+    oq, Sq = oracle_mod.quadratic(q, k, v, s0, phi=phi)
+    assert _rel(oq, ob) < 1e-12 and _rel(Sq, Sb) < 1e-12
