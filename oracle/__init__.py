@@ -14,7 +14,11 @@ What it computes (page "MiniMax-M1„ÅßÁêÜËß£„Åô„ÇãÔºöÂ§ßË¶èÊ®°Ë®ÄË™û„É¢„Éá„É´„ÅÆ„
   page "MiniMax: ¬´–ü–æ—á–µ–º—É M2 –≤ –∏—Ç–æ–≥–µ —Å—Ç–∞–ª–∞ –º–æ–¥–µ–ª—å—é —Å –ø–æ–ª–Ω—ã–º –≤–Ω–∏–º–∞–Ω–∏–µ–º?¬ª",
   section 1, glossary entry "Lightning Attention");
 * one decode step  S <- S + k v^T, o = q S                          (``decode``)
-* packed ragged batches with an optional resumed state per sequence (``varlen``).
+* packed ragged batches with an optional resumed state per sequence (``varlen``);
+* gradients of the recurrent form for given dO and dS_N (``backward``): the
+  chain rule through the recurrence, dq_t = do_t S_t^T, and with
+  G_t = sum_{t'>=t} q_t'^T do_t' + dS_N, dk_t = G_t v_t, dv_t = G_t^T k_t,
+  dS_0 = G_1.
 
 Every function takes ``phi`` (None / "identity", "elu1", "relu"): the
 element-wise feature map of the same page's phi(Q)(phi(K)^T V), applied in
@@ -65,6 +69,8 @@ def _load():
         lib.oracle_decode.restype = None
         lib.oracle_varlen.argtypes = [ctypes.c_int, ip] + [ctypes.c_int] * 3 + [dp] * 4 + [ip, dp, dp]
         lib.oracle_varlen.restype = None
+        lib.oracle_backward.argtypes = [ctypes.c_int] * 4 + [dp] * 10
+        lib.oracle_backward.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -157,3 +163,20 @@ def varlen(q, k, v, cu_seqlens, state_pool=None, init_idx=None, phi=None):
                           _ptr(pool), idx.ctypes.data_as(ip) if idx is not None else ip(),
                           _ptr(o), _ptr(s_out))
     return o, s_out
+
+
+def backward(q, k, v, do, s0=None, ds_n=None):
+    """Gradients (dq, dk, dv, ds0) of the dense recurrent form for dL/dO = do
+    and dL/dS_N = ds_n (zero if None); shapes as ``recurrent``."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    s0, ds_n = _f64(s0), _f64(ds_n)
+    *lead, N, d_k = q.shape
+    d_v = v.shape[-1]
+    assert k.shape == q.shape and v.shape == do.shape and tuple(v.shape[:-1]) == tuple(q.shape[:-1])
+    U = int(np.prod(lead)) if lead else 1
+    dq, dk = np.zeros_like(q), np.zeros_like(k)
+    dv = np.zeros_like(v)
+    ds0 = np.zeros(tuple(lead) + (d_k, d_v), np.float64)
+    _load().oracle_backward(U, N, d_k, d_v, _ptr(q), _ptr(k), _ptr(v), _ptr(s0), _ptr(do), _ptr(ds_n),
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds0))
+    return dq, dk, dv, ds0

@@ -182,3 +182,62 @@ void oracle_varlen(int n_seq, const int* cu, int H, int dk, int dv,
         free(S);
     }
 }
+
+/* Gradients of the dense recurrent form, by the chain rule through
+ *   S_t = S_{t-1} + k_t v_t^T (S_0 = s0),   o_t = q_t S_t,
+ * for a loss L with dL/do_t = do_t and dL/dS_N = ds_n (NULL = zero):
+ *   dq_t = do_t S_t^T                                   (forward sweep)
+ *   G_t  = sum_{t' >= t} q_t'^T do_t' + ds_n            (reverse sweep: the
+ *          gradient reaching k_t v_t^T through every later state)
+ *   dk_t = G_t v_t,   dv_t = G_t^T k_t,   ds0 = G_1.
+ * q,k,dq,dk [U][N][d_k]; v,do,dv [U][N][d_v]; s0, ds_n, ds0 [U][d_k][d_v]
+ * (s0, ds_n may be NULL = zero; ds0 may be NULL). */
+void oracle_backward(int U, int N, int d_k, int d_v,
+                     const double* q, const double* k, const double* v, const double* s0,
+                     const double* dout, const double* ds_n,
+                     double* dq, double* dk, double* dv, double* ds0) {
+    long sd = (long)d_k * d_v;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < U; ++u) {
+        const double* Q = q + (long)u * N * d_k;
+        const double* K = k + (long)u * N * d_k;
+        const double* V = v + (long)u * N * d_v;
+        const double* DO = dout + (long)u * N * d_v;
+        double* DQ = dq + (long)u * N * d_k;
+        double* DK = dk + (long)u * N * d_k;
+        double* DV = dv + (long)u * N * d_v;
+        double* S = (double*)malloc(sizeof(double) * (size_t)(sd > 0 ? sd : 1));
+        /* forward sweep: S_t, then dq_t = do_t S_t^T */
+        if (s0) memcpy(S, s0 + (long)u * sd, sizeof(double) * (size_t)sd);
+        else memset(S, 0, sizeof(double) * (size_t)sd);
+        for (int t = 0; t < N; ++t) {
+            for (int i = 0; i < d_k; ++i)
+                for (int j = 0; j < d_v; ++j) S[(long)i * d_v + j] += K[(long)t * d_k + i] * V[(long)t * d_v + j];
+            for (int i = 0; i < d_k; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d_v; ++j) acc += DO[(long)t * d_v + j] * S[(long)i * d_v + j];
+                DQ[(long)t * d_k + i] = acc;
+            }
+        }
+        /* reverse sweep: G_t, then dk_t = G_t v_t, dv_t = G_t^T k_t */
+        double* G = S;
+        if (ds_n) memcpy(G, ds_n + (long)u * sd, sizeof(double) * (size_t)sd);
+        else memset(G, 0, sizeof(double) * (size_t)sd);
+        for (int t = N - 1; t >= 0; --t) {
+            for (int i = 0; i < d_k; ++i)
+                for (int j = 0; j < d_v; ++j) G[(long)i * d_v + j] += Q[(long)t * d_k + i] * DO[(long)t * d_v + j];
+            for (int i = 0; i < d_k; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d_v; ++j) acc += G[(long)i * d_v + j] * V[(long)t * d_v + j];
+                DK[(long)t * d_k + i] = acc;
+            }
+            for (int j = 0; j < d_v; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < d_k; ++i) acc += G[(long)i * d_v + j] * K[(long)t * d_k + i];
+                DV[(long)t * d_v + j] = acc;
+            }
+        }
+        if (ds0) memcpy(ds0 + (long)u * sd, G, sizeof(double) * (size_t)sd);
+        free(S);
+    }
+}

@@ -365,3 +365,60 @@ def test_feature_map_enters_only_through_q_and_k(oracle_mod, phi):
     assert _rel(o, ob) < 1e-12 and _rel(S, Sb) < 1e-12
     oq, Sq = oracle_mod.quadratic(q, k, v, s0, phi=phi)
     assert _rel(oq, ob) < 1e-12 and _rel(Sq, Sb) < 1e-12
+
+
+# ------------------------------------------------------------------ backward
+
+def _loss(oracle_mod, q, k, v, s0, W, Z):
+    o, S = oracle_mod.recurrent(q, k, v, s0)
+    return float(np.sum(o * W) + np.sum(S * Z))
+
+
+def test_backward_matches_finite_differences(oracle_mod):
+    """Central differences of L = <O, W> + <S_N, Z> through the forward oracle;
+    dL/dO = W and dL/dS_N = Z are the backward's inputs."""
+    N, dk, dv = 5, 3, 4
+    q, k, v = _rand((N, dk), 51), _rand((N, dk), 52), _rand((N, dv), 53)
+    s0, W, Z = _rand((dk, dv), 54), _rand((N, dv), 55), _rand((dk, dv), 56)
+    dq, dk_, dv_, ds0 = oracle_mod.backward(q, k, v, W, s0, Z)
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk_), (v, dv_), (s0, ds0)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = [q, k, v, s0]
+            pos = [a is x for a in args].index(True)
+            ap, am = list(args), list(args)
+            ap[pos], am[pos] = xp, xm
+            num[idx] = (_loss(oracle_mod, *ap, W, Z) - _loss(oracle_mod, *am, W, Z)) / (2 * h)
+        assert _rel(g, num) < 1e-7
+
+
+def test_backward_matches_autograd_of_the_quadratic_form(oracle_mod):
+    """An independent derivation: torch autograd (float64, CPU) through the
+    masked quadratic form O = (Q K^T ⊙ M) V + Q S0, S_N = S0 + K^T V."""
+    import torch
+    N, dk, dv = 9, 4, 5
+    q, k, v = _rand((2, N, dk), 61), _rand((2, N, dk), 62), _rand((2, N, dv), 63)
+    s0, W, Z = _rand((2, dk, dv), 64), _rand((2, N, dv), 65), _rand((2, dk, dv), 66)
+    tq, tk, tv, ts0 = (torch.tensor(x, requires_grad=True) for x in (q, k, v, s0))
+    M = torch.tril(torch.ones(N, N, dtype=torch.float64))
+    O = ((tq @ tk.transpose(1, 2)) * M) @ tv + tq @ ts0
+    S = ts0 + tk.transpose(1, 2) @ tv
+    ((O * torch.tensor(W)).sum() + (S * torch.tensor(Z)).sum()).backward()
+    dq, dk_, dv_, ds0 = oracle_mod.backward(q, k, v, W, s0, Z)
+    for g, t in ((dq, tq), (dk_, tk), (dv_, tv), (ds0, ts0)):
+        assert _rel(g, t.grad.numpy()) < 1e-12
+
+
+def test_backward_single_token_closed_form(oracle_mod):
+    """N = 1, S0 = 0: o = (q.k) v, so dq = (do.v) k, dk = (do.v) q, dv = (q.k) do."""
+    q, k, v, do = _rand((1, 6), 71), _rand((1, 6), 72), _rand((1, 7), 73), _rand((1, 7), 74)
+    dq, dk_, dv_, ds0 = oracle_mod.backward(q, k, v, do)
+    a = float(do[0] @ v[0])
+    np.testing.assert_allclose(dq[0], a * k[0], rtol=1e-13)
+    np.testing.assert_allclose(dk_[0], a * q[0], rtol=1e-13)
+    np.testing.assert_allclose(dv_[0], float(q[0] @ k[0]) * do[0], rtol=1e-13)
+    np.testing.assert_allclose(ds0, np.outer(q[0], do[0]), rtol=1e-13)
