@@ -433,6 +433,29 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity"):
                 l2="inputs (1 GiB) larger than L2")
 
 
+def run_backward(args, dist: Dist, pk):
+    """Gradients of the 8K prefill (dq, dk, dv, ds0 for a given dO)."""
+    import long_context_linear_b200 as la
+    import synth
+    c = PREFILL8K
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=81 + dist.rank, device=dev)
+    _, _, do = synth.dense(B, H, N, d, "bf16", seed=91 + dist.rank, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = max(5, min(args.steps, 20))
+    total_ms, _ = timed_launches(lambda: la.prefill_backward(q, k, v, do), n, max(3, args.warmup), dist, stream)
+    ms_step = dist.max(total_ms) / n
+    # algorithmic bytes: q, k, v, dO read once, dq, dk, dv written once, ds0 written
+    byts = 7.0 * B * H * N * d * 2 + B * H * d * d * 4
+    gbs = byts / (ms_step / 1e3) / 1e9
+    del q, k, v, do
+    torch.cuda.empty_cache()
+    return dict(workload="backward of prefill B=4 H=32 N=8192 d=128 bf16 (FFMA kernel)",
+                tokens_per_s=B * N * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
+                frac=gbs / pk["hbm"], steps=n)
+
+
 def run_few_heads(args, dist: Dist, pk):
     """Long prefill with too few (batch, head) units to fill the GPU, once with
     the library's segment split and once with it turned off."""
@@ -570,6 +593,7 @@ def main():
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
         extras["few_heads"] = run_few_heads(args, dist, pk)
+        extras["backward_8k"] = run_backward(args, dist, pk)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_line()

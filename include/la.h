@@ -201,6 +201,31 @@ LA_API la_status la_decode_commit(const void* k, const void* v, float* S, const 
                                   la_stream_t stream);
 
 /*
+ * Gradients of la_prefill (dense layout, feature map identity): for a loss L
+ * with dL/dO = dout and dL/dS_N = ds_n, the chain rule through
+ * S_t = S_{t-1} + k_t (x) v_t, o_t = q_t S_t (page "MiniMax-M1で理解する…",
+ * section "線形アテンションの数学的基礎") gives
+ *   dq_t = dout_t S_t^T,   G_t = sum_{t' >= t} q_t'^T dout_t' + ds_n,
+ *   dk_t = G_t v_t,   dv_t = G_t^T k_t,   ds0 = G_1,
+ * computed chunk by chunk like the forward (masked products inside a chunk,
+ * S carried forward for dq and G carried backward for dk, dv).
+ *   q, k, dq, dk : [B, H, N, d_k];  v, dout, dv : [B, H, N, d_v]   dtype `dt`
+ *   s0, ds_n     : fp32 [B, H, d_k, d_v] or NULL (zero);  ds0: fp32 or NULL.
+ * bf16 with d = 128: three tensor-core passes of the prefill kernel
+ * (dq = prefill(dout, v, k) from s0^T; dk = prefill(v, dout, q) from ds_n^T
+ * and dv = prefill(k, q, dout) from ds_n, both with time reversed), with the
+ * prefill's precision.  fp32 or d = 64: one FFMA kernel, fp32 arithmetic.
+ * d_k = d_v in {64, 128}.  All pointers 16-byte aligned; the caller owns every
+ * buffer; no host synchronisation.  Errors: LA_ERR_INVALID_ARG (null, negative,
+ * misaligned), LA_ERR_UNSUPPORTED (dims), LA_ERR_CUDA (launch).
+ */
+LA_API la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout,
+                                     const float* s0, const float* ds_n,
+                                     void* dq, void* dk, void* dv, float* ds0,
+                                     int B, int H, int N, int d_k, int d_v, la_dtype dt,
+                                     la_stream_t stream);
+
+/*
  * Reads the device status word of the current device (synchronizes the
  * device).  *out receives LA_OK or LA_ERR_TIMEOUT; clear != 0 resets it.
  */

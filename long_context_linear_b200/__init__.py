@@ -19,7 +19,8 @@ import torch
 from . import _abi
 from ._abi import LAError, lib
 
-__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "decode_step", "decode_verify", "decode_commit",
+__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "prefill_backward", "decode_step", "decode_verify",
+           "decode_commit",
            "device_status", "LAError",
            "lib", "prefill_workspace_size", "prefill_varlen_workspace_size"]
 
@@ -103,6 +104,34 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torc
                                      _stream(q.device)),
                    "la_prefill_ex")
     return out, s_out
+
+
+def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,
+                     s0: Optional[torch.Tensor] = None, ds_n: Optional[torch.Tensor] = None, *,
+                     need_ds0: bool = True):
+    """Gradients of ``prefill`` for dL/dO = dout and dL/dS_N = ds_n (zero if None).
+
+    q, k, v, dout: [B, H, N, d]; s0, ds_n: fp32 [B, H, d, d] or None.
+    Returns (dq, dk, dv, ds0) with dq, dk, dv in the input dtype and ds0 fp32
+    (None unless need_ds0).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, n, q.dtype, q.device)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or dout.shape != v.shape:
+        raise ValueError("q, k, v, dout must all be [B, H, N, d]")
+    B, H, N, d = q.shape
+    for t, n in ((s0, "s0"), (ds_n, "ds_n")):
+        if t is not None:
+            _need(t, n, torch.float32, q.device)
+            if tuple(t.shape) != (B, H, d, d):
+                raise ValueError(f"{n} must be [B, H, d, d]")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds0 = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if need_ds0 else None
+    with torch.cuda.device(q.device):
+        _abi.check(lib.la_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(s0), _ptr(ds_n), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), _ptr(ds0), B, H, N, d, d, _dtype_code(q),
+                                           _stream(q.device)), "la_prefill_backward")
+    return dq, dk, dv, ds0
 
 
 def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,

@@ -26,6 +26,7 @@
 #include "selftest.cuh"
 #include "seg_prefix.cuh"
 #include "decode_multi.cuh"
+#include "backward_simt.cuh"
 
 namespace lcl {
 
@@ -141,10 +142,12 @@ la_status make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, u
     return LA_OK;
 }
 
-bool env_validate() {
-    const char* v = getenv("LA_VALIDATE");
+bool env_flag(const char* name) {
+    const char* v = getenv(name);
     return v && v[0] == '1';
 }
+
+bool env_validate() { return env_flag("LA_VALIDATE"); }
 
 la_status check_phi(la_phi phi) {
     if (phi != LA_PHI_IDENTITY && phi != LA_PHI_ELU1 && phi != LA_PHI_RELU)
@@ -213,6 +216,22 @@ void launch_decode(int dk, int grid, const void* q, const void* k, const void* v
     else
         dec::decode_step_kernel<T, SS, 64><<<grid, dec::NUM_THREADS, 0, st>>>(
             (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S, phi);
+}
+}  // namespace
+}  // namespace lcl
+
+namespace lcl {
+namespace {
+template <typename T, int D, int CS>
+la_status launch_backward(int grid, const void* q, const void* k, const void* v, const void* dout, void* dq,
+                          void* dk, void* dv, const bwd::Params& bp, cudaStream_t st) {
+    auto kern = bwd::backward_simt_kernel<T, D, CS>;
+    constexpr int smem = bwd::smem_bytes<D, CS>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (backward)");
+    kern<<<grid, bwd::NUM_THREADS, smem, st>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, (T*)dq, (T*)dk,
+                                                (T*)dv, bp);
+    return after_launch("backward launch");
 }
 }  // namespace
 }  // namespace lcl
@@ -624,6 +643,83 @@ extern "C" la_status la_prefill_varlen_noalloc(const void* q, const void* k, con
     if (s != LA_OK) return s;
     return la_prefill_varlen(q, k, v, o, cu_seqlens, n_seq, T, state_pool, n_pool, init_idx, s_out, H, dk, dv, dt,
                              chunk, scratch, sizeof(int) * LA_NOALLOC_MAX_SEQS, stream);
+}
+
+// One dense tensor-core pass over whole sequences: o = prefill(q, k, v) from
+// `init` (transposed if init_t), chunks visited last to first if `reverse`.
+la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
+                        float* s_out, bool reverse, long U, int N, int d, DeviceInfo* di, cudaStream_t st) {
+    if (N == 0 && !s_out) return LA_OK;
+    tc::Params p{};
+    p.mode = 0;
+    p.n_items = (int)(U * tc::NVS);
+    p.N = N;
+    p.dv = d;
+    p.s0 = init;
+    p.s_out = s_out;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.status = di->status;
+    p.n_seg = 1;
+    p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
+    p.phi = LA_PHI_IDENTITY;
+    p.reverse = reverse ? 1 : 0;
+    p.init_transposed = init_t ? 1 : 0;
+    const void* any = N > 0 ? q : s_out;
+    CUtensorMap mq, mk, mv, mo;
+    const uint64_t row = (uint64_t)d * 2, Nm = N > 0 ? (uint64_t)N : 1, unit = Nm * row;
+    la_status s;
+    if ((s = make_map(&mq, N > 0 ? q : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mk, N > 0 ? k : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mv, N > 0 ? v : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
+    if ((s = make_map(&mo, N > 0 ? o : any, d, Nm, U, row, unit, 32, 1)) != LA_OK) return s;
+    tc::prefill_tc_kernel<<<std::min(p.n_items, di->sms), tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    return after_launch("prefill_tc (backward pass) launch");
+}
+
+la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,
+                              const float* ds_n, void* dq, void* dk, void* dv, float* ds0, int B, int H, int N,
+                              int d_k, int d_v, la_dtype dt, la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(d_k, d_v, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || N < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d N=%d", B, H, N);
+    const long U = (long)B * H;
+    if (U > (1L << 29) || (long)N * U > (1L << 40)) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (U == 0) return LA_OK;
+    if (N > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv))
+        return fail(LA_ERR_INVALID_ARG, "q, k, v, dout, dq, dk, dv must be non-null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(s0) || !aligned16(ds_n) || !aligned16(ds0))
+        return fail(LA_ERR_INVALID_ARG, "all pointers must be 16-byte aligned");
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (use_tensor_cores(d_k, dt) && !env_flag("LA_BACKWARD_SIMT")) {
+        // Each gradient is a forward pass over permuted inputs (G_t is the
+        // suffix sum dS_N + sum_{t' >= t} q_t'^T do_t'):
+        //   dq_t = do_t S_t^T : prefill(dO, V, K) from s0^T
+        //   dk_t = v_t G_t^T  : prefill(V, dO, Q) from dS_N^T, chunks last to first
+        //   dv_t = k_t G_t    : prefill(K, Q, dO) from dS_N, chunks last to first;
+        //                       its final state is G_1 = dS_0
+        if (N > 0) {
+            if ((s = tc_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, di, st)) != LA_OK) return s;
+            if ((s = tc_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, di, st)) != LA_OK) return s;
+        }
+        return tc_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, di, st);
+    }
+    bwd::Params bp{};
+    bp.U = (int)U;
+    bp.N = N;
+    bp.s0 = s0;
+    bp.ds_n = ds_n;
+    bp.ds0 = ds0;
+    const int grid = (int)(2 * U);
+    if (d_k == 128) {
+        if (dt == LA_FP32) return launch_backward<float, 128, 32>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+        return launch_backward<__nv_bfloat16, 128, 32>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+    }
+    if (dt == LA_FP32) return launch_backward<float, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+    return launch_backward<__nv_bfloat16, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
 }
 
 la_status la_selftest_wait_timeout(int timeout_us, la_stream_t stream) {

@@ -113,6 +113,10 @@ struct Params {
     int s_out_per_seg;     // 1: s_out holds the state after every segment, [U][n_seg][DK][dv]
     int state_only;        // 1: only the state is computed (no Q, no outputs)
     int phi;               // feature map on q and k (phi.cuh); applied to the tiles in smem
+    // dense, one segment only: visit the chunks last to first and keep s >= t
+    // inside a chunk, so that o_t = q_t (S_init + sum_{s >= t} k_s v_s^T)
+    int reverse;
+    int init_transposed;   // the initial state is given as its transpose [dv][DK]
 };
 
 struct Item {
@@ -130,6 +134,9 @@ __device__ __forceinline__ int item_index(int round, int cta, int grid) {
     // arrive longest first
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
+
+// First token (relative to the item's start) of the c-th chunk in visiting order.
+__device__ __forceinline__ int chunk_row(const Params& p, int c, int nc) { return (p.reverse ? nc - 1 - c : c) * C; }
 
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     Item it;
@@ -321,7 +328,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int c = -PREFETCH; c < nc; ++c) {
                     const int cp = c + PREFETCH;
                     if (cp < nc) {
-                        const int y = p.mode == 0 ? it.t0 + cp * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + cp * C;
+                        const int t = it.t0 + chunk_row(p, cp, nc);
+                        const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
                         if (!p.state_only) {
                             tma_prefetch_3d(&map_q, 0, y, z);
                             tma_prefetch_3d(&map_q, 64, y, z);
@@ -331,7 +339,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         tma_prefetch_3d(&map_v, DVS * it.vs, y, z);
                     }
                     if (c < 0) continue;
-                    const int y = p.mode == 0 ? it.t0 + c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
+                    const int t = it.t0 + chunk_row(p, c, nc);
+                    const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
                     const int qs = g % Q_SLOTS, kq = g / Q_SLOTS;
                     if (!p.state_only) {
                         if (kq > 0 && !mbar_wait(&q_empty[qs], (kq - 1) & 1, abort, p.status)) { stop = true; break; }
@@ -366,7 +375,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const Item it = decode_item(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
-                    const int y = p.mode == 0 ? it.t0 + c * C : it.c1, z = p.mode == 0 ? it.c2 : it.t0 + c * C;
+                    const int t = it.t0 + chunk_row(p, c, nc);
+                    const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
                     const int vc = g % V_SLOTS, kv = g / V_SLOTS;
                     if (kv > 0 && !mbar_wait(&v_empty[vc], (kv - 1) & 1, abort, p.status)) { stop = true; break; }
                     mbar_arrive_expect_tx(&v_full[vc], PANEL);
@@ -423,7 +433,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     const int rows = len - c0;
                     const int ksteps = (p.mode == 1 && rows < C) ? (rows + 15) >> 4 : C / 16;
                     if (!mbar_wait(&p_ready[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
-                    if (ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
+                    if (p.mode == 1 && ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
                     tc_fence_after();
                     const uint32_t tpo = tbase + TM_PO_STRIDE * b;
                     const uint64_t dv = mnmaj_desc(sv + vc * PANEL, 0, PANEL);
@@ -464,7 +474,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     uint64_t* kready = p.phi != PHI_IDENTITY ? &kphi_full[ks] : &k_full[ks];
                     if (!mbar_wait(kready, (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                     if (!mbar_wait(&v_full[vc], (g / V_SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                    if (ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
+                    if (p.mode == 1 && ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
                     if (g >= 2 && !mbar_wait(&ds_empty[b], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
                     const uint32_t tds = tbase + TM_DS + TM_PO_STRIDE * b;
@@ -490,8 +500,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             // ------------------------------------------------------ mask warps
             // Row t = 32 q4 + lane of P; 32-column piece pc holds keys 32 pc ...
             // Pieces below the diagonal piece are kept whole, the diagonal piece
-            // keeps s <= t, pieces above it are zero.  bf16 piece pc goes to
-            // columns 16 pc .. 16 pc + 15, which only overlap fp32 pieces already read.
+            // keeps s <= t, pieces above it are zero (in reverse order: pieces
+            // above kept, s >= t on the diagonal, pieces below zero).  bf16
+            // piece pc goes to columns 16 pc .. 16 pc + 15, which only overlap
+            // fp32 pieces already read.
             const int q4 = warp & 3;
             int g = 0;
             bool stop = false;
@@ -507,15 +519,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 #pragma unroll 1
                     for (int pc = 0; pc < 4; ++pc) {
                         uint32_t pk[16];
-                        if (pc <= q4) {
+                        if (p.reverse ? pc >= q4 : pc <= q4) {
                             uint32_t v[32];
                             tmem_ld32(ta + 32 * pc, v);
                             tmem_wait_ld();
-                            const int keep = pc < q4 ? 31 : lane;  // last kept column within the piece
+                            // kept columns lo .. hi within the piece
+                            const int lo = (p.reverse && pc == q4) ? lane : 0;
+                            const int hi = (!p.reverse && pc == q4) ? lane : 31;
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
-                                pk[i] = pack_bf16x2(2 * i <= keep ? __uint_as_float(v[2 * i]) : 0.f,
-                                                    2 * i + 1 <= keep ? __uint_as_float(v[2 * i + 1]) : 0.f);
+                                pk[i] = pack_bf16x2((2 * i >= lo && 2 * i <= hi) ? __uint_as_float(v[2 * i]) : 0.f,
+                                                    (2 * i + 1 >= lo && 2 * i + 1 <= hi) ? __uint_as_float(v[2 * i + 1]) : 0.f);
                         } else {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) pk[i] = 0u;
@@ -547,7 +561,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             if (idx >= p.n_items) break;
             const Item it = decode_item(p, idx);
             float S[DVS];
-            if (it.init) {
+            if (it.init && p.init_transposed) {
+                // column i of rows DVS vs .. DVS vs + DVS - 1 of the transposed block
+                const float* src = it.init + (long)DVS * it.vs * DK + i;
+#pragma unroll
+                for (int j = 0; j < DVS; ++j) S[j] = src[j * DK];
+            } else if (it.init) {
                 const float4* src = reinterpret_cast<const float4*>(it.init + (long)i * p.dv + DVS * it.vs);
 #pragma unroll
                 for (int j = 0; j < DVS / 4; ++j) {
@@ -631,7 +650,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
                 const Item it = decode_item(p, idx);
-                for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
+                const int nc = (it.len + C - 1) / C;
+                for (int c = 0; c < nc; ++c, ++g) {
+                    const int c0 = chunk_row(p, c, nc);
                     const int b = g & 1;
                     if (!warp_wait(&o_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();

@@ -173,6 +173,17 @@ def test_prefill_ex_rejects_unknown_feature_map(lib):
     assert st == 1
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(dq=None), 1), (dict(q=FAKE + 4), 1), (dict(N=-1), 1), (dict(dk=32, dv=32), 2), (dict(dk=64, dv=128), 2)])
+def test_backward_rejects_bad_arguments(lib, kw, status):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, do=FAKE, s0=None, dsn=None, dq=FAKE, dkk=FAKE, dvv=FAKE, ds0=None, B=1, H=1,
+             N=8, dk=128, dv=128, dt=0, stream=None)
+    a.update(kw)
+    st = lib.la_prefill_backward(a["q"], a["k"], a["v"], a["do"], a["s0"], a["dsn"], a["dq"], a["dkk"], a["dvv"],
+                                 a["ds0"], a["B"], a["H"], a["N"], a["dk"], a["dv"], a["dt"], a["stream"])
+    assert st == status
+
+
 def test_device_status_null(lib):
     assert lib.la_device_status(None, 0) == 1
 
