@@ -416,15 +416,18 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity"):
     q, k, v = synth.dense(B, H, N, d, "bf16", seed=61 + dist.rank, device=dev)
     o = torch.empty_like(v)
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    # with phi != identity the workspace holds phi(q), phi(k) (mapped by a pre-pass)
+    ws_bytes = la.prefill_workspace_size(B, H, N, d, torch.bfloat16, phi)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     n = max(10, min(args.steps, 200))
-    total_ms, per = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, phi=phi), n,
+    total_ms, per = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, phi=phi, workspace=ws), n,
                                    max(3, args.warmup), dist, stream)
     total_ms = dist.max(total_ms)
     ms_step = total_ms / n
     byts = prefill_bytes(B, H, N, d)
     gbs = byts / (ms_step / 1e3) / 1e9
-    del q, k, v, o, s
+    del q, k, v, o, s, ws
     torch.cuda.empty_cache()
     return dict(workload=f"prefill B=4 H=32 N=8192 d=128 bf16, feature map {phi}",
                 tokens_per_s=B * N * dist.world / (ms_step / 1e3),

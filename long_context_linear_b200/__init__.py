@@ -59,12 +59,13 @@ def _need(t: torch.Tensor, name: str, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
-def prefill_workspace_size(B: int, H: int, N: int, d: int, dtype: torch.dtype) -> int:
-    return int(lib.la_prefill_workspace_size(B, H, N, d, d, _DT[dtype]))
+def prefill_workspace_size(B: int, H: int, N: int, d: int, dtype: torch.dtype, phi: str = "identity") -> int:
+    return int(lib.la_prefill_workspace_size_ex(B, H, N, d, d, _DT[dtype], _phi_code(phi)))
 
 
-def prefill_varlen_workspace_size(n_seq: int, T: int, H: int, d: int, dtype: torch.dtype) -> int:
-    return int(lib.la_prefill_varlen_workspace_size(n_seq, T, H, d, d, _DT[dtype]))
+def prefill_varlen_workspace_size(n_seq: int, T: int, H: int, d: int, dtype: torch.dtype,
+                                  phi: str = "identity") -> int:
+    return int(lib.la_prefill_varlen_workspace_size_ex(n_seq, T, H, d, d, _DT[dtype], _phi_code(phi)))
 
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torch.Tensor] = None, *,
@@ -94,7 +95,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torc
         s_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     if s_out is not None:
         _need(s_out, "s_out", torch.float32, q.device)
-    need = int(lib.la_prefill_workspace_size(B, H, N, dk, dv, dt))
+    need = int(lib.la_prefill_workspace_size_ex(B, H, N, dk, dv, dt, _phi_code(phi)))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -170,7 +171,7 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
         s_out = torch.empty((max(n_seq, 0), H, dk, dv), dtype=torch.float32, device=q.device)
     if s_out is not None:
         _need(s_out, "s_out", torch.float32, q.device)
-    need = int(lib.la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt))
+    need = int(lib.la_prefill_varlen_workspace_size_ex(n_seq, T, H, dk, dv, dt, _phi_code(phi)))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -34,6 +34,8 @@ SIGNATURES = {
     "la_last_error": (ctypes.c_char_p, []),
     "la_version": (_i, []),
     "la_prefill_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "la_prefill_workspace_size_ex": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "la_prefill_varlen_workspace_size_ex": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "la_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "la_prefill_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "la_prefill_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -66,7 +68,7 @@ class LAError(RuntimeError):
 def load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"CUDA library {LIB_PATH} is not built; run `python -m long_context_linear_b200.build` "
+            f"CUDA library {LIB_PATH} is not built; run `python long_context_linear_b200/build.py` "
             "(needs nvcc with sm_100a support). There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

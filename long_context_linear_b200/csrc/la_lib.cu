@@ -27,6 +27,7 @@
 #include "seg_prefix.cuh"
 #include "decode_multi.cuh"
 #include "backward_simt.cuh"
+#include "phi_map.cuh"
 
 namespace lcl {
 
@@ -286,15 +287,49 @@ size_t segment_workspace_bytes(long U, int P, int dk, int dv) {
     return (size_t)U * (size_t)(2 * P - 1) * (size_t)dk * (size_t)dv * sizeof(float);
 }
 
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Scratch for phi(q) and phi(k) (bf16, `rows` rows of d) on the tensor-core
+// path; zero for the identity.
+size_t phi_workspace_bytes(long rows, int d, la_phi phi) {
+    if (phi == LA_PHI_IDENTITY || rows <= 0) return 0;
+    return 2 * round256((size_t)rows * (size_t)d * 2);
+}
+
+// phi over q and k (each `elems` bf16) into the two halves of `scratch`; on
+// success q and k are redirected to the mapped copies.
+la_status phi_prepass(const void** q, const void** k, void* scratch, long elems, la_phi phi, DeviceInfo* di,
+                      cudaStream_t st) {
+    const long n = elems / 8;  // elems is a multiple of d = 128
+    uint8_t* yq = reinterpret_cast<uint8_t*>(scratch);
+    uint8_t* yk = yq + round256((size_t)elems * 2);
+    const long per_block = (long)phimap::NUM_THREADS * phimap::VPT;
+    const int blocks = (int)std::min<long>((2 * n + per_block - 1) / per_block, 8L * di->sms);
+    phimap::phi_map_kernel<<<blocks, phimap::NUM_THREADS, 0, st>>>(
+        reinterpret_cast<const uint4*>(*q), reinterpret_cast<const uint4*>(*k), reinterpret_cast<uint4*>(yq),
+        reinterpret_cast<uint4*>(yk), n, (int)phi);
+    la_status s = after_launch("phi pre-pass launch");
+    if (s != LA_OK) return s;
+    *q = yq;
+    *k = yk;
+    return LA_OK;
+}
+
 }  // namespace
 
 size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt) {
+    return la_prefill_workspace_size_ex(B, H, N, dk, dv, dt, LA_PHI_IDENTITY);
+}
+
+size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtype dt, la_phi phi) {
     if (B <= 0 || H <= 0 || N <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return 0;
-    DeviceInfo* di;
-    if (device_info(&di) != LA_OK) return 0;
-    int seg_len;
     const long U = (long)B * H;
-    return segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), dk, dv);
+    const size_t ph = phi_workspace_bytes(U * N, dk, phi);
+    DeviceInfo* di;
+    if (device_info(&di) != LA_OK) return ph;
+    int seg_len;
+    const size_t seg = segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), dk, dv);
+    return ph ? round256(seg) + ph : seg;
 }
 
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
@@ -353,6 +388,15 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         P = 1;  // no room for the segment states: one pass over whole sequences
         p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
     }
+    // phi(q), phi(k) mapped up front when the workspace has room behind the
+    // segment states; otherwise the kernel maps the tiles in shared memory
+    const size_t off_phi = P > 1 ? round256(ws_need) : 0, ws_phi = phi_workspace_bytes(U * N, dk, phi);
+    if (ws_phi && workspace && aligned16(workspace) && ws_bytes >= off_phi + ws_phi) {
+        if ((s = phi_prepass(&q, &k, reinterpret_cast<uint8_t*>(workspace) + off_phi, U * N * dk, phi, di, st)) !=
+            LA_OK)
+            return s;
+        p.phi = LA_PHI_IDENTITY;
+    }
     // With N = 0 no tile is ever copied; the maps then only need a valid base.
     const void* bq = N > 0 ? q : s_out;
     const void* bk = N > 0 ? k : s_out;
@@ -397,7 +441,13 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
 size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt) {
     (void)T; (void)H; (void)dk; (void)dv; (void)dt;
     if (n_seq <= 0) return 0;
-    return ((size_t)n_seq * sizeof(int) + 255) & ~(size_t)255;
+    return round256((size_t)n_seq * sizeof(int));
+}
+
+size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int dv, la_dtype dt, la_phi phi) {
+    const size_t base = la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt);
+    if (!base || T <= 0 || H <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return base;
+    return base + phi_workspace_bytes((long)T * H, dk, phi);
 }
 
 la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
@@ -467,6 +517,13 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     int* order = reinterpret_cast<int*>(workspace);
     vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
     if ((s = after_launch("varlen order launch")) != LA_OK) return s;
+    const size_t ws_phi = T > 0 ? phi_workspace_bytes((long)T * H, dk, phi) : 0;
+    if (ws_phi && ws_bytes >= need + ws_phi) {
+        if ((s = phi_prepass(&q, &k, reinterpret_cast<uint8_t*>(workspace) + need, (long)T * H * dk, phi, di, st)) !=
+            LA_OK)
+            return s;
+        phi = LA_PHI_IDENTITY;
+    }
 
     tc::Params p{};
     p.mode = 1;

@@ -11,9 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from long_context_linear_b200 import build
-    build.build()
-    from long_context_linear_b200 import _abi
+    from long_context_linear_b200 import _abi  # built by conftest at session start
     return _abi.lib
 
 
@@ -52,6 +50,19 @@ def test_workspace_sizes(lib):
     assert lib.la_prefill_varlen_workspace_size(0, 0, 32, 128, 128, 0) == 0
     ws = lib.la_prefill_varlen_workspace_size(64, 10 ** 6, 32, 128, 128, 0)
     assert ws >= 64 * 4 and ws % 256 == 0
+
+
+def test_workspace_sizes_with_feature_map(lib):
+    # identity adds nothing; elu+1 / relu add phi(q) and phi(k) in bf16 on the tensor-core path
+    assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, 0) == 0
+    for phi in (1, 2):
+        assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, phi) == 2 * 4 * 32 * 8192 * 128 * 2
+        assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 1, phi) == 0  # fp32: mapped at load
+        base = lib.la_prefill_varlen_workspace_size(64, 1000, 32, 128, 128, 0)
+        assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, phi) == base + 2 * 1000 * 32 * 256
+        assert lib.la_prefill_varlen_workspace_size_ex(64, 1001, 3, 128, 128, 0, phi) == base + 2 * (
+            (1001 * 3 * 256 + 255) // 256 * 256)
+    assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, 0) == base
 
 
 FAKE = 1 << 20  # a 16-byte aligned non-null "device pointer"; never dereferenced on these paths

@@ -122,3 +122,62 @@ def test_unknown_phi_is_rejected(la):
     q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError):
         la.prefill(q, q, q, phi="tanh")
+
+
+def _raw_prefill(la, q, k, v, phi, ws):
+    """la_prefill_ex through the C ABI with the given (possibly too small) workspace."""
+    B, H, N, d = q.shape
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=q.device)
+    wsb = 0 if ws is None else ws.numel()
+    st = la.lib.la_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, s.data_ptr(), B, H, N,
+                              d, d, 0, 0, la.PHI[phi], None if ws is None else ws.data_ptr(), wsb,
+                              torch.cuda.current_stream().cuda_stream)
+    assert st == 0, la.lib.la_last_error()
+    return o, s
+
+
+@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("segments", [None, "3"])
+def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, phi, segments):
+    """With room in the workspace q and k are mapped by a pre-pass; without it
+    the kernel maps the tiles in shared memory.  Both round phi to bf16 the
+    same way, so the results are bit-identical."""
+    if segments:
+        monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N = 1, 2, 3000
+    q, k, v = synth.dense(B, H, N, 128, "bf16", seed=91, device="cuda")
+    full = la.prefill_workspace_size(B, H, N, 128, torch.bfloat16, phi)
+    seg = la.prefill_workspace_size(B, H, N, 128, torch.bfloat16)
+    assert full >= seg + 2 * B * H * N * 128 * 2
+    ws_full = torch.empty(full, dtype=torch.uint8, device="cuda")
+    ws_seg = torch.empty(seg, dtype=torch.uint8, device="cuda") if seg else None
+    o1, s1 = _raw_prefill(la, q, k, v, phi, ws_full)
+    o2, s2 = _raw_prefill(la, q, k, v, phi, ws_seg)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    assert torch.equal(o1, o2)
+    assert torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_varlen_phi_prepass_equals_in_kernel_mapping(la, phi):
+    lens = [700, 1, 129, 2000]
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
+    T, H, d = int(cu[-1]), 3, 128
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=5, device="cuda")
+    outs = []
+    for with_phi_room in (True, False):
+        n = la.prefill_varlen_workspace_size(len(lens), T, H, d, torch.bfloat16, phi if with_phi_room else "identity")
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+        o = torch.empty_like(v)
+        s = torch.empty(len(lens), H, d, d, dtype=torch.float32, device="cuda")
+        st = la.lib.la_prefill_varlen_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), cu.data_ptr(),
+                                         len(lens), T, None, 0, None, s.data_ptr(), H, d, d, 0, 0, la.PHI[phi],
+                                         ws.data_ptr(), n, torch.cuda.current_stream().cuda_stream)
+        assert st == 0, la.lib.la_last_error()
+        outs.append((o, s))
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
