@@ -523,13 +523,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                             uint32_t v[32];
                             tmem_ld32(ta + 32 * pc, v);
                             tmem_wait_ld();
-                            // kept columns lo .. hi within the piece
-                            const int lo = (p.reverse && pc == q4) ? lane : 0;
-                            const int hi = (!p.reverse && pc == q4) ? lane : 31;
+                            // bit j: column j of the piece is kept
+                            const uint32_t keep = pc != q4 ? 0xffffffffu
+                                                           : (p.reverse ? 0xffffffffu << lane : 0xffffffffu >> (31 - lane));
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
-                                pk[i] = pack_bf16x2((2 * i >= lo && 2 * i <= hi) ? __uint_as_float(v[2 * i]) : 0.f,
-                                                    (2 * i + 1 >= lo && 2 * i + 1 <= hi) ? __uint_as_float(v[2 * i + 1]) : 0.f);
+                                pk[i] = pack_bf16x2((keep & (1u << (2 * i))) ? __uint_as_float(v[2 * i]) : 0.f,
+                                                    (keep & (2u << (2 * i))) ? __uint_as_float(v[2 * i + 1]) : 0.f);
                         } else {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) pk[i] = 0u;
