@@ -102,7 +102,9 @@ la_status device_info(DeviceInfo** out) {
             return cuda_fail(e, "cudaDeviceGetAttribute");
         if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word)) != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress");
-        if ((e = cudaFuncSetAttribute(tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(tc::prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      tc::SMEM_BYTES)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(tc::prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       tc::SMEM_BYTES)) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
         if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
@@ -180,6 +182,16 @@ la_status after_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, what);
     return LA_OK;
+}
+
+// The tensor-core prefill, lean instance unless an option needs the general one.
+la_status launch_tc(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
+    const bool general =
+        p.phi != LA_PHI_IDENTITY || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1);
+    if (general) tc::prefill_tc_kernel<true><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    else tc::prefill_tc_kernel<false><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    return after_launch(what);
 }
 
 template <typename T, int D>
@@ -422,9 +434,9 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         p1.s_out = seg_sums;
         p1.s_out_per_seg = 1;
         p1.state_only = 1;
-        tc::prefill_tc_kernel<<<std::min(p1.n_items, di->sms), tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv,
-                                                                                                   mo, p1);
-        if ((s = after_launch("prefill_tc (segment sums) launch")) != LA_OK) return s;
+        if ((s = launch_tc(std::min(p1.n_items, di->sms), mq, mk, mv, mo, p1, st, "prefill_tc (segment sums) launch")) !=
+            LA_OK)
+            return s;
         const long threads = U * (long)(dk * dv / 4);
         const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
         segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(seg_sums, s0, starts, U, P, dk * dv);
@@ -434,8 +446,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         p.seg_init = starts;
     }
     const int grid = std::min(p.n_items, di->sms);
-    tc::prefill_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
-    return after_launch("prefill_tc launch");
+    return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc launch");
 }
 
 size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt) {
@@ -548,8 +559,7 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     if ((s = make_map(&mv, v ? v : any, dv, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
     if ((s = make_map(&mo, o ? o : any, dv, H, Tm, head, tok, 1, 32)) != LA_OK) return s;
     const int grid = std::min(p.n_items, di->sms);
-    tc::prefill_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
-    return after_launch("prefill_tc (varlen) launch");
+    return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc (varlen) launch");
 }
 
 la_status la_decode_step_ex(const void* q, const void* k, const void* v, void* o, void* S, int B, int H, int dk,
@@ -729,8 +739,7 @@ la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, co
     if ((s = make_map(&mk, N > 0 ? k : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mv, N > 0 ? v : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mo, N > 0 ? o : any, d, Nm, U, row, unit, 32, 1)) != LA_OK) return s;
-    tc::prefill_tc_kernel<<<std::min(p.n_items, di->sms), tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
-    return after_launch("prefill_tc (backward pass) launch");
+    return launch_tc(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_tc (backward pass) launch");
 }
 
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,

@@ -136,12 +136,23 @@ __device__ __forceinline__ int item_index(int round, int cta, int grid) {
 }
 
 // First token (relative to the item's start) of the c-th chunk in visiting order.
-__device__ __forceinline__ int chunk_row(const Params& p, int c, int nc) { return (p.reverse ? nc - 1 - c : c) * C; }
+__device__ __forceinline__ int chunk_row(bool rev, int c, int nc) { return (rev ? nc - 1 - c : c) * C; }
 
+// kGeneral = false: dense items are whole sequences (n_seg = 1).
+template <bool kGeneral>
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     Item it;
     it.vs = idx & (NVS - 1);
-    if (p.mode == 0) {
+    if (!kGeneral && p.mode == 0) {
+        const int u = idx / NVS;
+        it.t0 = 0;
+        it.len = p.N;
+        it.c1 = 0;
+        it.c2 = u;
+        it.state = u;
+        it.init = p.s0 ? p.s0 + (long)u * DK * p.dv : nullptr;
+        it.write_state = true;
+    } else if (p.mode == 0) {
         const int us = idx / NVS;  // unit * n_seg + segment
         const int u = us / p.n_seg, sg = us - u * p.n_seg;
         it.t0 = sg * p.seg_len;
@@ -239,6 +250,11 @@ __device__ __forceinline__ constexpr uint64_t mnmaj_step(int kk) { return static
 // The code below is kept compact on purpose: all warps of all SMs run their
 // roles' loops at once, so the kernel's instruction footprint (not only its
 // instruction count) decides how often warps stall on instruction fetch.
+// kGeneral = false is the lean instance for the common case (feature map
+// identity, chunks in order, outputs computed, initial state as given, whole
+// sequences): the options below are then compile-time constants and their
+// code is left out.
+template <bool kGeneral>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -270,6 +286,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int lane = threadIdx.x & 31;
     const int G = gridDim.x;
     const int cta = blockIdx.x;
+    const bool state_only = kGeneral && p.state_only;
+    const int phi = kGeneral ? p.phi : static_cast<int>(PHI_IDENTITY);
+    const bool rev = kGeneral && p.reverse;
+    const bool init_t = kGeneral && p.init_transposed;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < Q_SLOTS; ++i) {
@@ -279,12 +299,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         for (int i = 0; i < K_SLOTS; ++i) {
             mbar_init(&kphi_full[i], 4);
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], p.state_only ? 1 : 2);
+            mbar_init(&k_empty[i], state_only ? 1 : 2);
             mbar_init(&s_full[i], 4);
         }
         for (int i = 0; i < V_SLOTS; ++i) {
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], p.state_only ? 1 : 2);
+            mbar_init(&v_empty[i], state_only ? 1 : 2);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&p_full[i], 1);
@@ -322,15 +342,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item(p, idx);
+                const Item it = decode_item<kGeneral>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 // chunk c is brought into L2 PREFETCH chunks before its load
                 for (int c = -PREFETCH; c < nc; ++c) {
                     const int cp = c + PREFETCH;
                     if (cp < nc) {
-                        const int t = it.t0 + chunk_row(p, cp, nc);
+                        const int t = it.t0 + chunk_row(rev, cp, nc);
                         const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
-                        if (!p.state_only) {
+                        if (!state_only) {
                             tma_prefetch_3d(&map_q, 0, y, z);
                             tma_prefetch_3d(&map_q, 64, y, z);
                         }
@@ -339,10 +359,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         tma_prefetch_3d(&map_v, DVS * it.vs, y, z);
                     }
                     if (c < 0) continue;
-                    const int t = it.t0 + chunk_row(p, c, nc);
+                    const int t = it.t0 + chunk_row(rev, c, nc);
                     const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
                     const int qs = g % Q_SLOTS, kq = g / Q_SLOTS;
-                    if (!p.state_only) {
+                    if (!state_only) {
                         if (kq > 0 && !mbar_wait(&q_empty[qs], (kq - 1) & 1, abort, p.status)) { stop = true; break; }
                         uint8_t* qb = sm + OFF_Q + qs * TILE_Q;
                         mbar_arrive_expect_tx(&q_full[qs], TILE_Q);
@@ -360,7 +380,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
             // make sure no copy into shared memory is still in flight at exit
             for (int x = (g >= Q_SLOTS ? g - Q_SLOTS : 0); x < g; ++x) {
-                if (!p.state_only) drain_wait(&q_full[x % Q_SLOTS], (x / Q_SLOTS) & 1);
+                if (!state_only) drain_wait(&q_full[x % Q_SLOTS], (x / Q_SLOTS) & 1);
                 drain_wait(&k_full[x % K_SLOTS], (x / K_SLOTS) & 1);
             }
         }
@@ -372,10 +392,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item(p, idx);
+                const Item it = decode_item<kGeneral>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
-                    const int t = it.t0 + chunk_row(p, c, nc);
+                    const int t = it.t0 + chunk_row(rev, c, nc);
                     const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
                     const int vc = g % V_SLOTS, kv = g / V_SLOTS;
                     if (kv > 0 && !mbar_wait(&v_empty[vc], (kv - 1) & 1, abort, p.status)) { stop = true; break; }
@@ -392,7 +412,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // P V of chunk g, so its mask runs while P V and the next product are
         // queued.  TMEM written or read by other warps is ordered by
         // tcgen05.fence::after_thread_sync after the barrier.
-        if (lane == 0 && !p.state_only) {
+        if (lane == 0 && !state_only) {
             constexpr uint32_t id_f = idesc_bf16(128, C + DVS, 0, 0);  // Q [K ; S^T]^T
             constexpr uint32_t id_pv = idesc_bf16(128, DVS, 0, 1);     // P V (P from TMEM)
             const uint32_t sq = smem_u32(sm + OFF_Q), sk = smem_u32(sm + OFF_K), sv = smem_u32(sm + OFF_V);
@@ -400,7 +420,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0;; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                total += (decode_item(p, idx).len + C - 1) / C;
+                total += (decode_item<kGeneral>(p, idx).len + C - 1) / C;
             }
             int k = 0;  // next chunk whose [P|O] is to be issued
             int g = 0;  // chunk whose P V is issued next
@@ -408,7 +428,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item(p, idx).len;
+                const int len = decode_item<kGeneral>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     // [P | O] = Q [K ; S^T]^T for chunks up to g + 1  (A: Q, B: K rows then S^T rows)
                     for (; k <= g + 1 && k < total; ++k) {
@@ -465,13 +485,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item(p, idx).len;
+                const int len = decode_item<kGeneral>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     const int ks = g % K_SLOTS, vc = g % V_SLOTS, b = g & 1;
                     const int rows = len - c0;
                     const int ksteps = (p.mode == 1 && rows < C) ? (rows + 15) >> 4 : C / 16;
                     // dS = K^T V   (A: K MN-major over 2 panels, B: V MN-major)
-                    uint64_t* kready = p.phi != PHI_IDENTITY ? &kphi_full[ks] : &k_full[ks];
+                    uint64_t* kready = phi != PHI_IDENTITY ? &kphi_full[ks] : &k_full[ks];
                     if (!mbar_wait(kready, (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                     if (!mbar_wait(&v_full[vc], (g / V_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                     if (p.mode == 1 && ksteps * 16 > rows) clear_tail_rows(sm + OFF_V + vc * PANEL, rows, ksteps);
@@ -496,7 +516,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         __syncwarp();
     } else if (warp < 6) {
-        if (!p.state_only) {
+        if (!state_only) {
             // ------------------------------------------------------ mask warps
             // Row t = 32 q4 + lane of P; 32-column piece pc holds keys 32 pc ...
             // Pieces below the diagonal piece are kept whole, the diagonal piece
@@ -510,7 +530,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item(p, idx).len;
+                const int len = decode_item<kGeneral>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     const int b = g & 1;
                     if (!warp_wait(&p_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
@@ -519,13 +539,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 #pragma unroll 1
                     for (int pc = 0; pc < 4; ++pc) {
                         uint32_t pk[16];
-                        if (p.reverse ? pc >= q4 : pc <= q4) {
+                        if (rev ? pc >= q4 : pc <= q4) {
                             uint32_t v[32];
                             tmem_ld32(ta + 32 * pc, v);
                             tmem_wait_ld();
                             // bit j: column j of the piece is kept
                             const uint32_t keep = pc != q4 ? 0xffffffffu
-                                                           : (p.reverse ? 0xffffffffu << lane : 0xffffffffu >> (31 - lane));
+                                                           : (rev ? 0xffffffffu << lane : 0xffffffffu >> (31 - lane));
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
                                 pk[i] = pack_bf16x2((keep & (1u << (2 * i))) ? __uint_as_float(v[2 * i]) : 0.f,
@@ -559,9 +579,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         for (int r = 0; !stop; ++r) {
             const int idx = item_index(r, cta, G);
             if (idx >= p.n_items) break;
-            const Item it = decode_item(p, idx);
+            const Item it = decode_item<kGeneral>(p, idx);
             float S[DVS];
-            if (it.init && p.init_transposed) {
+            if (it.init && init_t) {
                 // column i of rows DVS vs .. DVS vs + DVS - 1 of the transposed block
                 const float* src = it.init + (long)DVS * it.vs * DK + i;
 #pragma unroll
@@ -580,7 +600,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
                 // publish bf16(S_{c-1})^T next to K_c, once the slot's previous product is done
                 const int ks = g % K_SLOTS;
-                if (!p.state_only) {
+                if (!state_only) {
                     if (g >= K_SLOTS && !warp_wait(&k_empty[ks], ((g / K_SLOTS) - 1) & 1, abort, p.status)) { stop = true; break; }
                     uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
                     __nv_bfloat16* rowp[8];
@@ -594,21 +614,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     // buffer it writes (last used by chunk c - 2) drained
                     if (!warp_wait(&q_full[g % Q_SLOTS], (g / Q_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                 }
-                if (p.phi != PHI_IDENTITY || !p.state_only) {
+                if (phi != PHI_IDENTITY || !state_only) {
                     if (!warp_wait(&k_full[ks], (g / K_SLOTS) & 1, abort, p.status)) { stop = true; break; }
                 }
-                if (p.phi != PHI_IDENTITY) {
+                if (phi != PHI_IDENTITY) {
                     // phi(K_c), then phi(Q_c), in place, before the tensor cores read
                     // them (the S^T rows behind K are left alone); K first, so that
                     // K^T V can start while Q is mapped
-                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, 2 * PANEL / 16, i, p.phi);
+                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, 2 * PANEL / 16, i, phi);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&kphi_full[ks]);
-                    if (!p.state_only)
+                    if (!state_only)
                         phi_region(smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q), PANEL, PANEL / 16, 2 * PANEL / 16, i,
-                                   p.phi);
+                                   phi);
                 }
-                if (!p.state_only) {
+                if (!state_only) {
                     if (g >= 2 && !warp_wait(&o_empty[g & 1], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
                     tc_fence_before();
@@ -639,7 +659,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
         }
     } else if (warp < 14) {
-        if (!p.state_only) {
+        if (!state_only) {
             // ------------------------------------------------------ output warps
             const int q4 = warp & 3;
             const int row = q4 * 32 + lane;
@@ -649,10 +669,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item(p, idx);
+                const Item it = decode_item<kGeneral>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
-                    const int c0 = chunk_row(p, c, nc);
+                    const int c0 = chunk_row(rev, c, nc);
                     const int b = g & 1;
                     if (!warp_wait(&o_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
