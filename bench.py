@@ -50,8 +50,8 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "2bf09d47bbe89457"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.73e6 + 115.07e6) / (16 * 32768)
+TRAFFIC_HASH = "2f86a51311fbd1f4"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.71e6 + 117.04e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
@@ -454,7 +454,7 @@ def run_backward(args, dist: Dist, pk):
     gbs = byts / (ms_step / 1e3) / 1e9
     del q, k, v, do
     torch.cuda.empty_cache()
-    return dict(workload="backward of prefill B=4 H=32 N=8192 d=128 bf16 (FFMA kernel)",
+    return dict(workload="backward of prefill B=4 H=32 N=8192 d=128 bf16 (three tensor-core passes)",
                 tokens_per_s=B * N * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
                 frac=gbs / pk["hbm"], steps=n)
 
