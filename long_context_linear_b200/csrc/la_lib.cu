@@ -235,6 +235,20 @@ void launch_decode(int dk, int grid, const void* q, const void* k, const void* v
 
 namespace lcl {
 namespace {
+template <typename T, int D>
+void launch_commit_d(int m, int grid, const T* k, const T* v, float* S, const int32_t* accepted, int H, int phi,
+                     cudaStream_t st) {
+    if (m > 8) dmulti::commit_kernel<T, D, 3><<<grid, dmulti::NUM_THREADS, 0, st>>>(k, v, S, accepted, H, m, phi);
+    else dmulti::commit_kernel<T, D, 2><<<grid, dmulti::NUM_THREADS, 0, st>>>(k, v, S, accepted, H, m, phi);
+}
+
+template <typename T>
+void launch_commit(int dk, int m, int grid, const void* k, const void* v, float* S, const int32_t* accepted, int H,
+                   int phi, cudaStream_t st) {
+    if (dk == 128) launch_commit_d<T, 128>(m, grid, (const T*)k, (const T*)v, S, accepted, H, phi, st);
+    else launch_commit_d<T, 64>(m, grid, (const T*)k, (const T*)v, S, accepted, H, phi, st);
+}
+
 template <typename T, int D, int CS>
 la_status launch_backward(int grid, const void* q, const void* k, const void* v, const void* dout, void* dq,
                           void* dk, void* dv, const bwd::Params& bp, cudaStream_t st) {
@@ -656,15 +670,8 @@ la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t
             if (h[b] < 0 || h[b] > m) return fail(LA_ERR_INVALID_ARG, "accepted[%d]=%d outside 0..%d", b, h[b], m);
     }
     const int grid = (int)U;
-    if (dt == LA_BF16) {
-        using T = __nv_bfloat16;
-        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
-        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
-    } else {
-        using T = float;
-        if (dk == 128) dmulti::commit_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
-        else dmulti::commit_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)k, (const T*)v, S, accepted, H, m, phi);
-    }
+    if (dt == LA_BF16) launch_commit<__nv_bfloat16>(dk, m, grid, k, v, S, accepted, H, phi, st);
+    else launch_commit<float>(dk, m, grid, k, v, S, accepted, H, phi, st);
     return after_launch("decode_commit launch");
 }
 

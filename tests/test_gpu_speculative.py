@@ -64,12 +64,13 @@ def test_commit_matches_recurrence_over_accepted_prefix(la, oracle_mod, m):
         assert_state(got[b:b + 1], rs, 2, tol=1e-6)
 
 
-def test_commit_equals_decode_steps_bit_for_bit(la):
+@pytest.mark.parametrize("m,acc", [(6, [0, 2, 5, 6]), (12, [1, 9, 12, 0])])  # both commit instances (m <= 8, m > 8)
+def test_commit_equals_decode_steps_bit_for_bit(la, m, acc):
     """Commit adds the accepted tokens with one fused multiply-add each, in
     token order, exactly as consecutive decode steps do."""
-    B, H, m, d = 4, 2, 6, 128
-    S, q, k, v = _case(B, H, m, d, "bf16", seed=7)
-    accepted = torch.tensor([0, 2, 5, 6], dtype=torch.int32)
+    B, H, d = 4, 2, 128
+    S, q, k, v = _case(B, H, m, d, "bf16", seed=7 + m)
+    accepted = torch.tensor(acc, dtype=torch.int32)
     S_commit = S.cuda()
     la.decode_commit(k.cuda(), v.cuda(), S_commit, accepted.cuda())
     for b in range(B):
