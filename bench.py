@@ -312,7 +312,8 @@ def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
     gbs = bytes_step / (ms_step / 1e3) / 1e9
     del S, qs, ks, vs, os_
     torch.cuda.empty_cache()
-    name = {torch.float32: "fp32", torch.bfloat16: "bf16", torch.float16: "fp16"}[state_dtype]
+    name = {torch.float32: "fp32", torch.bfloat16: "bf16", torch.float16: "fp16",
+            torch.float8_e4m3fn: "fp8_e4m3", torch.float8_e5m2: "fp8_e5m2"}[state_dtype]
     return dict(workload=f"decode B=256 H=64 d=128 bf16 q/k/v, {name} state, 1024 consecutive steps",
                 hbm_gbs=gbs, peak_gbs=pk["hbm"], frac=gbs / pk["hbm"], ms_per_step=ms_step,
                 bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
@@ -591,6 +592,7 @@ def main():
         # state stored in bf16 / fp16, updated in fp32 (the low-precision storage study)
         extras["decode_bf16_state"] = run_decode(args, dist, pk, torch.bfloat16)
         extras["decode_fp16_state"] = run_decode(args, dist, pk, torch.float16)
+        extras["decode_fp8_e4m3_state"] = run_decode(args, dist, pk, torch.float8_e4m3fn)
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)

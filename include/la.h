@@ -64,7 +64,13 @@ typedef enum {
 typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
 
 /* Storage format of a decode state (see la_decode_step_ex). */
-typedef enum { LA_STATE_FP32 = 0, LA_STATE_BF16 = 1, LA_STATE_FP16 = 2 } la_state_dtype;
+typedef enum {
+    LA_STATE_FP32 = 0,
+    LA_STATE_BF16 = 1,
+    LA_STATE_FP16 = 2,
+    LA_STATE_FP8_E4M3 = 3, /* 8-bit, 3 mantissa bits, largest finite 448 (no infinities) */
+    LA_STATE_FP8_E5M2 = 4  /* 8-bit, 2 mantissa bits, largest finite 57344 */
+} la_state_dtype;
 
 /*
  * Element-wise feature map phi on queries and keys.  Page "MiniMax-M1で理解す
@@ -177,10 +183,11 @@ LA_API la_status la_decode_step(const void* q, const void* k, const void* v, voi
  * and page "ノーフリーランチ：MiniMax M2が高効率アテンション機構を解体",
  * infrastructure section, warn about (the state is rewritten at every token,
  * so its rounding errors accumulate).
- *   S: [B, H, d, d] in `sdt` (fp32, bf16 or fp16), updated IN PLACE.
- *   Each element is updated in fp32 as RN_fp32(S + k_i v_j) (one fused
- *   multiply-add) and rounded to `sdt` to nearest even; o = q S uses the
- *   stored, rounded state.  LA_STATE_FP32 is exactly la_decode_step.
+ *   S: [B, H, d, d] in `sdt` (fp32, bf16, fp16, fp8 e4m3 or fp8 e5m2),
+ *   updated IN PLACE.  Each element is updated in fp32 as RN_fp32(S + k_i v_j)
+ *   (one fused multiply-add) and rounded to `sdt` to nearest even (the 8-bit
+ *   formats saturate at their largest finite value); o = q S uses the stored,
+ *   rounded state.  LA_STATE_FP32 is exactly la_decode_step.
  *   Low-precision storage needs bf16 q, k, v (LA_ERR_UNSUPPORTED otherwise).
  *   phi (see la_phi) is applied to q and k as they are loaded.
  */

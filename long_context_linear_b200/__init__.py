@@ -213,21 +213,23 @@ def prefill_varlen_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu
 
 
 _STATE_DT = {torch.float32: _abi.LA_STATE_FP32, torch.bfloat16: _abi.LA_STATE_BF16,
-             torch.float16: _abi.LA_STATE_FP16}
+             torch.float16: _abi.LA_STATE_FP16, torch.float8_e4m3fn: _abi.LA_STATE_FP8_E4M3,
+             torch.float8_e5m2: _abi.LA_STATE_FP8_E5M2}
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, S: torch.Tensor, *,
                 out: Optional[torch.Tensor] = None, phi: str = "identity") -> torch.Tensor:
     """One token per (batch, head): S <- S + k (x) v in place, returns o = q S.
 
-    q, k, v: [B, H, d]; S: [B, H, d, d] in fp32, or in bf16 / fp16 (state
-    stored in low precision, updated in fp32 and rounded to nearest even;
-    needs bf16 q, k, v).
+    q, k, v: [B, H, d]; S: [B, H, d, d] in fp32, or in bf16 / fp16 /
+    float8_e4m3fn / float8_e5m2 (state stored in low precision, updated in fp32
+    and rounded to nearest even, the 8-bit formats saturating at their largest
+    finite value; needs bf16 q, k, v).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype, q.device)
     if S.dtype not in _STATE_DT:
-        raise TypeError(f"S must be float32, bfloat16 or float16, got {S.dtype}")
+        raise TypeError(f"S must be float32, bfloat16, float16, float8_e4m3fn or float8_e5m2, got {S.dtype}")
     _need(S, "S", S.dtype, q.device)
     if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
         raise ValueError("q, k must be [B, H, dk] and v [B, H, dv]")

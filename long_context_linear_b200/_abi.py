@@ -21,6 +21,8 @@ LA_FP32 = 1
 LA_STATE_FP32 = 0
 LA_STATE_BF16 = 1
 LA_STATE_FP16 = 2
+LA_STATE_FP8_E4M3 = 3
+LA_STATE_FP8_E5M2 = 4
 LA_PHI_IDENTITY = 0
 LA_PHI_ELU1 = 1
 LA_PHI_RELU = 2

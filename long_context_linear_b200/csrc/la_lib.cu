@@ -224,10 +224,10 @@ template <typename T, typename SS>
 void launch_decode(int dk, int grid, const void* q, const void* k, const void* v, void* o, void* S, int phi,
                    cudaStream_t st) {
     if (dk == 128)
-        dec::decode_step_kernel<T, SS, 128><<<grid, dec::NUM_THREADS, 0, st>>>(
+        dec::decode_step_kernel<T, SS, 128><<<grid, dec::decode_threads<SS>(), 0, st>>>(
             (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S, phi);
     else
-        dec::decode_step_kernel<T, SS, 64><<<grid, dec::NUM_THREADS, 0, st>>>(
+        dec::decode_step_kernel<T, SS, 64><<<grid, dec::decode_threads<SS>(), 0, st>>>(
             (const T*)q, (const T*)k, (const T*)v, (T*)o, (SS*)S, phi);
 }
 }  // namespace
@@ -582,7 +582,8 @@ la_status la_decode_step_ex(const void* q, const void* k, const void* v, void* o
     la_status s = check_dims(dk, dv, dt);
     if (s != LA_OK) return s;
     if ((s = check_phi(phi)) != LA_OK) return s;
-    if (sdt != LA_STATE_FP32 && sdt != LA_STATE_BF16 && sdt != LA_STATE_FP16)
+    if (sdt != LA_STATE_FP32 && sdt != LA_STATE_BF16 && sdt != LA_STATE_FP16 && sdt != LA_STATE_FP8_E4M3 &&
+        sdt != LA_STATE_FP8_E5M2)
         return fail(LA_ERR_INVALID_ARG, "unknown state dtype %d", (int)sdt);
     if (sdt != LA_STATE_FP32 && dt != LA_BF16)
         return fail(LA_ERR_UNSUPPORTED, "a bf16 or fp16 state needs bf16 q, k, v");
@@ -603,8 +604,12 @@ la_status la_decode_step_ex(const void* q, const void* k, const void* v, void* o
         launch_decode<__nv_bfloat16, float>(dk, grid, q, k, v, o, S, phi, st);
     } else if (sdt == LA_STATE_BF16) {
         launch_decode<__nv_bfloat16, __nv_bfloat16>(dk, grid, q, k, v, o, S, phi, st);
-    } else {
+    } else if (sdt == LA_STATE_FP16) {
         launch_decode<__nv_bfloat16, __half>(dk, grid, q, k, v, o, S, phi, st);
+    } else if (sdt == LA_STATE_FP8_E4M3) {
+        launch_decode<__nv_bfloat16, __nv_fp8_e4m3>(dk, grid, q, k, v, o, S, phi, st);
+    } else {
+        launch_decode<__nv_bfloat16, __nv_fp8_e5m2>(dk, grid, q, k, v, o, S, phi, st);
     }
     return after_launch("decode_step launch");
 }

@@ -15,7 +15,9 @@ storage" means for one decode step of S_t = S_{t-1} + k_t v_t^T, o_t = q_t S_t
 * every state element is updated in fp32: s = RN_fp32(S_stored + k_i v_j)
   (for bf16 inputs the product k_i v_j has at most 16 significant bits and is
   exact in fp32, so this is one fp32 addition of the exact product);
-* the result is rounded to the storage format (bf16 or fp16) to nearest even;
+* the result is rounded to the storage format (bf16, fp16, or the 8-bit
+  formats e4m3 / e5m2) to nearest even; the 8-bit formats saturate to their
+  largest finite value (448 / 57344) instead of overflowing;
 * o = q S uses the stored, rounded state (computed here in float64).
 
 Because the stored state is a rounding decision taken in fp32 on both sides, a
@@ -28,7 +30,13 @@ from typing import Tuple
 
 import numpy as np
 
-FORMATS = ("fp32", "bf16", "fp16")
+FORMATS = ("fp32", "bf16", "fp16", "fp8_e4m3", "fp8_e5m2")
+
+# 8-bit floating-point formats: (mantissa bits, exponent of the smallest
+# normal value, largest finite value).  e4m3: bias 7, no infinities, the
+# all-ones code is NaN, so the largest finite value is 1.75 * 2^8; e5m2: bias
+# 15, IEEE-like, largest finite 1.75 * 2^15.
+FP8 = {"fp8_e4m3": (3, -6, 448.0), "fp8_e5m2": (2, -14, 57344.0)}
 
 
 def round_bf16(x) -> np.ndarray:
@@ -45,7 +53,25 @@ def round_fp16(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float32).astype(np.float16).astype(np.float32)
 
 
+def round_fp8(x, fmt: str) -> np.ndarray:
+    """float32 values rounded to an 8-bit format (``FP8``) to nearest even,
+    saturating at the largest finite value, returned as float32.  Finite
+    inputs only.  Below the smallest normal value the spacing stays that of
+    the smallest binade (subnormals)."""
+    mant, emin, vmax = FP8[fmt]
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(a)                          # a = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, emin)                 # binade of a (or the subnormal range)
+    quantum = np.ldexp(1.0, e - mant)            # spacing of representable values there
+    r = np.round(a / quantum) * quantum          # a / quantum is exact; np.round is half-to-even
+    r = np.minimum(r, vmax)
+    return (np.sign(x) * r).astype(np.float32)
+
+
 def round_to(x, fmt: str) -> np.ndarray:
+    if fmt in FP8:
+        return round_fp8(x, fmt)
     if fmt == "fp32":
         return np.asarray(x, dtype=np.float32)
     if fmt == "bf16":

@@ -142,9 +142,10 @@ def _decode_state(lib, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(sdt=3), 1), (dict(sdt=-1), 1),   # unknown storage format
+    (dict(sdt=5), 1), (dict(sdt=-1), 1),   # unknown storage format
     (dict(dt=1, sdt=1), 2),                # a bf16 state needs bf16 inputs
-    (dict(dt=1, sdt=2), 2),                # ... as does an fp16 state
+    (dict(dt=1, sdt=2), 2),                # ... as do fp16 and fp8 states
+    (dict(dt=1, sdt=3), 2), (dict(dt=1, sdt=4), 2),
     (dict(S=None), 1), (dict(S=FAKE + 8), 1), (dict(B=-1), 1), (dict(dk=64, dv=128), 2),
     (dict(phi=3), 1), (dict(phi=-1), 1)])
 def test_decode_state_rejects_bad_arguments(lib, kw, status):

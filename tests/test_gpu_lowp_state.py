@@ -1,4 +1,4 @@
-"""Decode with the state stored in bf16 / fp16 (updated in fp32), through the C ABI.
+"""Decode with the state stored in bf16 / fp16 / fp8 (updated in fp32), through the C ABI.
 
 Parity: the stored state is a rounding decision taken in fp32 on both sides,
 so the GPU state must equal oracle/lowp.py's bit for bit after every step; o
@@ -16,7 +16,8 @@ from tests.parity import assert_out
 
 pytestmark = pytest.mark.gpu
 
-TORCH_FMT = {"fp32": torch.float32, "bf16": torch.bfloat16, "fp16": torch.float16}
+TORCH_FMT = {"fp32": torch.float32, "bf16": torch.bfloat16, "fp16": torch.float16,
+             "fp8_e4m3": torch.float8_e4m3fn, "fp8_e5m2": torch.float8_e5m2}
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +26,7 @@ def la():
     return la
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "fp16", "fp32"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp16", "fp32", "fp8_e4m3", "fp8_e5m2"])
 @pytest.mark.parametrize("d", [64, 128])
 def test_lowp_state_matches_oracle_bit_for_bit(la, fmt, d):
     from oracle import lowp
@@ -33,7 +34,8 @@ def test_lowp_state_matches_oracle_bit_for_bit(la, fmt, d):
     U = B * H
     L = [2000 + 500 * u for u in range(U)]
     S32 = synth.outer_product_state(U, d, d, L, seed=17).view(B, H, d, d)
-    S = S32.to(TORCH_FMT[fmt]).cuda()                  # the stored starting state
+    # the stored starting state, rounded by the oracle's rule
+    S = torch.from_numpy(lowp.round_to(S32.numpy(), fmt)).to(TORCH_FMT[fmt]).cuda()
     S_ref = S.float().cpu().numpy()
     qs, ks, vs = synth.qkv((T, B, H, d), d, "bf16", seed=19)
     for t in range(T):
@@ -48,7 +50,8 @@ def test_lowp_state_matches_oracle_bit_for_bit(la, fmt, d):
 def test_lowp_state_drift_over_steps(la, oracle_mod):
     """Relative Frobenius error of the stored state against the exact fp64
     recurrence after T steps, from states built from 16K-token prefixes.  fp32
-    storage stays at rounding level, fp16 and bf16 drift, bf16 the most."""
+    storage stays at rounding level; fp16, bf16 and the 8-bit formats drift,
+    the more the fewer mantissa bits they keep."""
     B, H, d = 4, 8, 128
     U = B * H
     steps = (64, 512, 2048)
@@ -72,7 +75,11 @@ def test_lowp_state_drift_over_steps(la, oracle_mod):
     for f in TORCH_FMT:
         print(f"  {f}: start {start_err[f]:.2e}  " + "  ".join(f"T={t}: {err[f][t]:.2e}" for t in steps))
     assert err["fp32"][steps[-1]] < 1e-6
-    assert err["fp32"][steps[-1]] < err["fp16"][steps[-1]] < err["bf16"][steps[-1]]
+    final = {f: err[f][steps[-1]] for f in TORCH_FMT}
+    # fewer mantissa bits, more drift: 23 > 10 > 7 > 3 > 2
+    assert final["fp32"] < final["fp16"] < final["bf16"] < final["fp8_e4m3"] < final["fp8_e5m2"]
     # storage rounding accumulates: the drift grows with the number of rewrites
     for f in ("fp16", "bf16"):
         assert err[f][steps[-1]] > err[f][steps[0]] > start_err[f]
+    for f in ("fp8_e4m3", "fp8_e5m2"):
+        assert err[f][steps[-1]] > err[f][steps[0]]

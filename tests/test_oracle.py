@@ -297,6 +297,69 @@ def test_lowp_fp16_rounding_follows_the_format_definition():
     np.testing.assert_array_equal(lowp.round_fp16(x), want)
 
 
+def _fp8_code_values(fmt):
+    """Every finite value of an 8-bit format, decoded from its bit fields:
+    sign | exponent (4 or 5 bits) | mantissa (3 or 2 bits).  e4m3: bias 7, the
+    code with all exponent and mantissa bits set is NaN, no infinities; e5m2:
+    bias 15, exponent all ones is infinity / NaN."""
+    eb, mb, bias = (4, 3, 7) if fmt == "fp8_e4m3" else (5, 2, 15)
+    vals = []
+    for code in range(256):
+        sign = -1.0 if code >> 7 else 1.0
+        ef = (code >> mb) & ((1 << eb) - 1)
+        mf = code & ((1 << mb) - 1)
+        if fmt == "fp8_e4m3" and ef == 15 and mf == 7:
+            continue
+        if fmt == "fp8_e5m2" and ef == 31:
+            continue
+        if ef == 0:
+            v = mf * 2.0 ** (1 - bias - mb)                       # subnormal
+        else:
+            v = (1 + mf / 2.0 ** mb) * 2.0 ** (ef - bias)
+        vals.append((sign * v, mf))
+    return vals
+
+
+@pytest.mark.parametrize("fmt,vmax,tiny", [("fp8_e4m3", 448.0, 2.0**-9), ("fp8_e5m2", 57344.0, 2.0**-16)])
+def test_lowp_fp8_rounding_follows_the_format_definition(fmt, vmax, tiny):
+    """Checked against every code of the format: representable values are kept,
+    the midpoint of two neighbours goes to the one with the even mantissa field,
+    values beyond the largest finite one saturate."""
+    from oracle import lowp
+    vals = _fp8_code_values(fmt)
+    pos = sorted({v: mf for v, mf in vals if v >= 0}.items())
+    values = np.array([v for v, _ in vals], dtype=np.float32)
+    np.testing.assert_array_equal(lowp.round_fp8(values, fmt), values)
+    assert pos[-1][0] == vmax and pos[1][0] == tiny
+    lo = np.array([a for (a, _), _ in zip(pos[:-1], pos[1:])])
+    hi = np.array([b for _, (b, _) in zip(pos[:-1], pos[1:])])
+    even_hi = np.array([mb % 2 == 0 for _, (_, mb) in zip(pos[:-1], pos[1:])])
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)   # midpoints are exact in fp32
+    want = np.where(even_hi, hi, lo).astype(np.float32)
+    np.testing.assert_array_equal(lowp.round_fp8(mid, fmt), want)
+    np.testing.assert_array_equal(lowp.round_fp8(-mid, fmt), -want)
+    # just below / above a midpoint: the nearer neighbour
+    np.testing.assert_array_equal(lowp.round_fp8(np.nextafter(mid, np.float32(0)), fmt), lo.astype(np.float32))
+    np.testing.assert_array_equal(lowp.round_fp8(np.nextafter(mid, np.float32(np.inf)), fmt), hi.astype(np.float32))
+    big = np.array([vmax * 1.01, vmax * 4, 1e30, -1e30], dtype=np.float32)
+    np.testing.assert_array_equal(lowp.round_fp8(big, fmt), np.array([vmax, vmax, vmax, -vmax], dtype=np.float32))
+
+
+@pytest.mark.parametrize("fmt,dtype", [("fp8_e4m3", "float8_e4m3fn"), ("fp8_e5m2", "float8_e5m2")])
+def test_lowp_fp8_rounding_matches_the_library_cast_in_range(fmt, dtype):
+    """Against torch's float8 cast (round to nearest even) on values inside the
+    finite range, where saturation plays no part."""
+    import torch
+    from oracle import lowp
+    rng = np.random.default_rng(11)
+    vmax = lowp.FP8[fmt][2]
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-4, 1e-2, 1.0, 30.0, vmax / 8)])
+    x = x[np.abs(x) < vmax].astype(np.float32)
+    want = torch.from_numpy(x).to(getattr(torch, dtype)).float().numpy()
+    np.testing.assert_array_equal(lowp.round_fp8(x, fmt), want)
+
+
 @pytest.mark.parametrize("fmt", ["fp32", "bf16", "fp16"])
 def test_lowp_decode_is_exact_where_the_format_holds_every_value(oracle_mod, fmt):
     """Integer inputs with |S| <= 64: every product, sum and stored value is
@@ -322,8 +385,16 @@ def test_lowp_decode_loses_updates_below_half_an_ulp():
     from oracle import lowp
     q = np.zeros(1)
     k, v = np.ones(1), np.full(1, 0.5)
-    for fmt, want in (("bf16", 256.0), ("fp16", 261.0), ("fp32", 261.0)):
+    for fmt, want in (("bf16", 256.0), ("fp16", 261.0), ("fp32", 261.0), ("fp8_e4m3", 256.0), ("fp8_e5m2", 256.0)):
         S = np.full((1, 1), 256.0, dtype=np.float32)
+        for _ in range(10):
+            _, S = lowp.decode_lowp(q, k, v, S, fmt)
+        assert S[0, 0] == want, (fmt, S[0, 0])
+    # from 4 with +0.5 per step: e4m3 (spacing 0.5 in [4, 8), 1 in [8, 16))
+    # climbs to 8, where 8.5 ties to the even 8 and stays; e5m2 (spacing 1 in
+    # [4, 8)) ties 4.5 to the even 4 at once; the wider formats reach 9
+    for fmt, want in (("fp8_e4m3", 8.0), ("fp8_e5m2", 4.0), ("bf16", 9.0), ("fp16", 9.0), ("fp32", 9.0)):
+        S = np.full((1, 1), 4.0, dtype=np.float32)
         for _ in range(10):
             _, S = lowp.decode_lowp(q, k, v, S, fmt)
         assert S[0, 0] == want, (fmt, S[0, 0])
