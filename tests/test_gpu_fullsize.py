@@ -117,3 +117,54 @@ def test_varlen_64_sequences_with_resume(la, oracle_mod):
         assert_state(s[n][hs].cpu(), rs, 1)
     del q, k, v, o, s, pool
     _free()
+
+
+def test_backward_b4_h32_n8192(la, oracle_mod):
+    """The gradients at the 8K prefill shape (three tensor-core passes), sampled
+    units against the oracle's chain rule."""
+    B, H, N, d = 4, 32, 8192, 128
+    dev = torch.device("cuda")
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=81, device=dev)
+    _, _, do = synth.dense(B, H, N, d, "bf16", seed=91, device=dev)
+    ds_n = torch.randn(B, H, d, d, device=dev, generator=torch.Generator(device=dev).manual_seed(93))
+    dq, dk, dv, ds0 = la.prefill_backward(q, k, v, do, None, ds_n)
+    assert la.device_status() == 0
+    units = synth.choose(B * H, 6, seed=6)
+    idx = torch.tensor(units, device=dev)
+    flat = lambda x: x.view(B * H, *x.shape[2:])[idx].cpu()  # noqa: E731
+    rq, rk, rv, rs0 = oracle_mod.backward(flat(q), flat(k), flat(v), flat(do), None, flat(ds_n))
+    for g, r in ((dq, rq), (dk, rk), (dv, rv)):
+        assert_out(flat(g), r, torch.bfloat16, 1)
+    assert_state(flat(ds0), rs0, 1)
+    del q, k, v, do, dq, dk, dv, ds0
+    _free()
+
+
+def test_speculative_b256_h64_m4(la, oracle_mod):
+    """Verify and commit of 4 drafts at the decode shape, sampled units against
+    the fp64 recurrence over the drafts."""
+    B, H, d, m = 256, 64, 128, 4
+    dev = torch.device("cuda")
+    U = B * H
+    g = torch.Generator(device=dev).manual_seed(97)
+    S = torch.randn(B, H, d, d, device=dev, generator=g) * 8.0   # the magnitude of a 8K-token state
+    q, k, v = synth.qkv((B, H, m, d), d, "bf16", seed=99, device=dev)
+    accepted = torch.randint(0, m + 1, (B,), generator=g, device=dev, dtype=torch.int32)
+    units = synth.choose(U, 32, seed=8)
+    idx = torch.tensor(units, device=dev)
+    S_before = S.view(U, d, d)[idx].cpu()
+    o = la.decode_verify(q, k, v, S)
+    la.decode_commit(k, v, S, accepted)
+    assert la.device_status() == 0
+    qf, kf, vf, of = (x.view(U, m, d)[idx].cpu() for x in (q, k, v, o))
+    ro, _ = oracle_mod.recurrent(qf, kf, vf, S_before)
+    assert_out(of, ro, torch.bfloat16, 1)
+    for j, u in enumerate(units):
+        a = int(accepted[u // H])
+        if a == 0:
+            assert torch.equal(S.view(U, d, d)[u].cpu(), S_before[j])
+            continue
+        _, rs = oracle_mod.recurrent(qf[j:j + 1, :a], kf[j:j + 1, :a], vf[j:j + 1, :a], S_before[j:j + 1])
+        assert_state(S.view(U, d, d)[u:u + 1].cpu(), rs, 1, tol=1e-6)
+    del S, q, k, v, o
+    _free()
