@@ -219,6 +219,28 @@ LA_API la_status la_decode_commit(const void* k, const void* v, float* S, const 
                                   la_stream_t stream);
 
 /*
+ * la_prefill on host-resident data: q, k, v, o (and s0, s_out) are HOST
+ * buffers in the la_prefill layout; page-locked memory lets the copies run
+ * asynchronously and overlap (pageable memory works, slower).  The (batch,
+ * head) units are processed in groups of `group`: while group i is computed
+ * on `stream`, group i + 1 is copied in and group i - 1 copied out on two
+ * internal copy streams, so host-to-device and device-to-host traffic run at
+ * the same time and the prefill itself hides under them.  Each group runs
+ * the single-pass kernel (no segment split), so the results equal those of
+ * la_prefill without a workspace bit for bit.
+ *   workspace: device scratch of at least la_prefill_host_workspace_size(...)
+ *   bytes (two staging buffers of `group` units each), 16-byte aligned.
+ * Asynchronous like every other call: `stream` is ordered after the last
+ * copy out, so synchronising it (or any later work on it) sees o and s_out.
+ * Errors: LA_ERR_INVALID_ARG (null, negative, group <= 0, workspace too
+ * small), LA_ERR_UNSUPPORTED (dims), LA_ERR_CUDA (copy or launch).
+ */
+LA_API size_t la_prefill_host_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt, int group);
+LA_API la_status la_prefill_host(const void* q, const void* k, const void* v, void* o,
+                                 const float* s0, float* s_out, int B, int H, int N, int dk, int dv,
+                                 la_dtype dt, int group, void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
  * Gradients of la_prefill (dense layout, feature map identity): for a loss L
  * with dL/dO = dout and dL/dS_N = ds_n, the chain rule through
  * S_t = S_{t-1} + k_t (x) v_t, o_t = q_t S_t (page "MiniMax-M1で理解する…",

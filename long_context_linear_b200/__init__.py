@@ -19,7 +19,8 @@ import torch
 from . import _abi
 from ._abi import LAError, lib
 
-__all__ = ["prefill", "prefill_varlen", "prefill_varlen_noalloc", "prefill_backward", "decode_step", "decode_verify",
+__all__ = ["prefill", "prefill_host", "prefill_varlen", "prefill_varlen_noalloc", "prefill_backward", "decode_step",
+           "decode_verify",
            "decode_commit",
            "device_status", "LAError",
            "lib", "prefill_workspace_size", "prefill_varlen_workspace_size"]
@@ -57,6 +58,15 @@ def _need(t: torch.Tensor, name: str, dtype=None, device=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if device is not None and t.device != device:
         raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _need_host(t: torch.Tensor, name: str, dtype=None):
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
 def prefill_workspace_size(B: int, H: int, N: int, d: int, dtype: torch.dtype, phi: str = "identity") -> int:
@@ -104,6 +114,48 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torc
                                      B, H, N, dk, dv, dt, chunk, _phi_code(phi), _ptr(workspace), ws_bytes,
                                      _stream(q.device)),
                    "la_prefill_ex")
+    return out, s_out
+
+
+def prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional[torch.Tensor] = None, *,
+                 group: int = 8, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
+                 return_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                 device: Optional[torch.device] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``prefill`` on host tensors (page-locked for overlap): q, k, v [B, H, N, d]
+    and s0 [B, H, d, d] fp32 on the CPU; returns host (O, S_N).
+
+    Groups of ``group`` (batch, head) units are copied in, computed and copied
+    out on overlapping streams of ``device`` (default: the current CUDA
+    device).  Asynchronous: synchronise that device's current stream before
+    reading the results.
+    """
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_host(t, n, q.dtype)
+    if q.dim() != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B, H, N, dk] and v [B, H, N, dv]")
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    pin = torch.cuda.is_available()
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, pin_memory=pin)
+    _need_host(out, "out", q.dtype)
+    if s0 is not None:
+        _need_host(s0, "s0", torch.float32)
+        if tuple(s0.shape) != (B, H, dk, dv):
+            raise ValueError("s0 must be [B, H, dk, dv]")
+    if s_out is None and return_state:
+        s_out = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=pin)
+    if s_out is not None:
+        _need_host(s_out, "s_out", torch.float32)
+    need = int(lib.la_prefill_host_workspace_size(B, H, N, dk, dv, dt, group))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _abi.check(lib.la_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(s0), _ptr(s_out), B, H, N, dk, dv,
+                                       dt, group, _ptr(workspace), ws_bytes, _stream(dev)), "la_prefill_host")
     return out, s_out
 
 

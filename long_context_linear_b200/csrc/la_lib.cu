@@ -63,6 +63,9 @@ struct DeviceInfo {
     int sms = 0;
     int* status = nullptr;       // device address of g_status_word
     bool attrs_set = false;
+    // copy streams of la_prefill_host, created on first use and kept for the
+    // life of the process (like a library handle)
+    cudaStream_t h2d = nullptr, d2h = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -798,6 +801,106 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
     }
     if (dt == LA_FP32) return launch_backward<float, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
     return launch_backward<__nv_bfloat16, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+}
+
+size_t la_prefill_host_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt, int group) {
+    if (B <= 0 || H <= 0 || N < 0 || group <= 0 || dk <= 0 || dv <= 0) return 0;
+    const size_t esz = dt == LA_FP32 ? 4 : 2;
+    const long g = std::min<long>(group, (long)B * H);
+    const size_t tok = round256((size_t)g * N * dk * esz) * 2 + round256((size_t)g * N * dv * esz) * 2;
+    const size_t st = round256((size_t)g * dk * dv * 4) * 2;
+    return 2 * (tok + st);  // two staging buffers
+}
+
+la_status la_prefill_host(const void* q, const void* k, const void* v, void* o, const float* s0, float* s_out, int B,
+                          int H, int N, int dk, int dv, la_dtype dt, int group, void* workspace, size_t ws_bytes,
+                          la_stream_t stream) {
+    g_last_error[0] = 0;
+    la_status s = check_dims(dk, dv, dt);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || N < 0) return fail(LA_ERR_INVALID_ARG, "negative size B=%d H=%d N=%d", B, H, N);
+    if (group <= 0) return fail(LA_ERR_INVALID_ARG, "group = %d must be positive", group);
+    const long U = (long)B * H;
+    if (U == 0) return LA_OK;
+    if (U > (1L << 30) || (long)N * U > (1L << 40)) return fail(LA_ERR_INVALID_ARG, "problem too large");
+    if (N > 0 && (!q || !k || !v || !o)) return fail(LA_ERR_INVALID_ARG, "q, k, v, o must be non-null");
+    const size_t need = la_prefill_host_workspace_size(B, H, N, dk, dv, dt, group);
+    if (!workspace || ws_bytes < need || !aligned16(workspace))
+        return fail(LA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu", need, ws_bytes);
+    DeviceInfo* di;
+    if ((s = device_info(&di)) != LA_OK) return s;
+    cudaError_t e = cudaSuccess;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        if (!di->h2d && (e = cudaStreamCreateWithFlags(&di->h2d, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithFlags");
+        if (!di->d2h && (e = cudaStreamCreateWithFlags(&di->d2h, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithFlags");
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long g = std::min<long>(group, U);
+    const size_t esz = dt == LA_FP32 ? 4 : 2;
+    const size_t qk_b = round256((size_t)g * N * dk * esz), vo_b = round256((size_t)g * N * dv * esz);
+    const size_t s_b = round256((size_t)g * dk * dv * 4);
+    const size_t buf_b = 2 * qk_b + 2 * vo_b + 2 * s_b;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    // events: start, then per staging buffer "copied in", "computed", "copied out"
+    cudaEvent_t ev[7] = {};
+    for (int i = 0; i < 7 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;
+    auto cleanup = [&]() {
+        for (int i = 0; i < 7; ++i)
+            if (ev[i]) cudaEventDestroy(ev[i]);
+    };
+    auto cu = [&](cudaError_t x, const char* what) -> la_status {
+        if (x == cudaSuccess) return LA_OK;
+        cleanup();
+        return cuda_fail(x, what);
+    };
+    if (e != cudaSuccess) return cu(e, "cudaEventCreate");
+    // the copy streams start after the work already queued on the caller's stream
+    if ((s = cu(cudaEventRecord(ev_start, st), "cudaEventRecord")) != LA_OK) return s;
+    if ((s = cu(cudaStreamWaitEvent(di->h2d, ev_start, 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+    if ((s = cu(cudaStreamWaitEvent(di->d2h, ev_start, 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+    const auto H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
+    for (long u0 = 0, i = 0; u0 < U; u0 += g, ++i) {
+        const int b = (int)(i & 1);
+        const long n = std::min(g, U - u0);
+        uint8_t* base = ws + b * buf_b;
+        uint8_t *dq = base, *dk_ = dq + qk_b, *dv_ = dk_ + qk_b, *do_ = dv_ + vo_b, *ds0 = do_ + vo_b, *dso = ds0 + s_b;
+        const size_t qk_n = (size_t)n * N * dk * esz, vo_n = (size_t)n * N * dv * esz, s_n = (size_t)n * dk * dv * 4;
+        const size_t qk_off = (size_t)u0 * N * dk * esz, vo_off = (size_t)u0 * N * dv * esz;
+        const size_t s_off = (size_t)u0 * dk * dv;
+        // buffer b is free once group i - 2 has been copied out
+        if (i >= 2 && (s = cu(cudaStreamWaitEvent(di->h2d, ev_out[b], 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+        if (qk_n) {
+            if ((s = cu(cudaMemcpyAsync(dq, (const uint8_t*)q + qk_off, qk_n, H2D, di->h2d), "copy q")) != LA_OK ||
+                (s = cu(cudaMemcpyAsync(dk_, (const uint8_t*)k + qk_off, qk_n, H2D, di->h2d), "copy k")) != LA_OK ||
+                (s = cu(cudaMemcpyAsync(dv_, (const uint8_t*)v + vo_off, vo_n, H2D, di->h2d), "copy v")) != LA_OK)
+                return s;
+        }
+        if (s0 && (s = cu(cudaMemcpyAsync(ds0, s0 + s_off, s_n, H2D, di->h2d), "copy s0")) != LA_OK) return s;
+        if ((s = cu(cudaEventRecord(ev_in[b], di->h2d), "cudaEventRecord")) != LA_OK) return s;
+        if ((s = cu(cudaStreamWaitEvent(st, ev_in[b], 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+        s = la_prefill_ex(dq, dk_, dv_, do_, s0 ? (const float*)ds0 : nullptr, s_out ? (float*)dso : nullptr, 1,
+                          (int)n, N, dk, dv, dt, 0, LA_PHI_IDENTITY, nullptr, 0, stream);
+        if (s != LA_OK) {
+            cleanup();
+            return s;
+        }
+        if ((s = cu(cudaEventRecord(ev_comp[b], st), "cudaEventRecord")) != LA_OK) return s;
+        if ((s = cu(cudaStreamWaitEvent(di->d2h, ev_comp[b], 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+        if (vo_n && (s = cu(cudaMemcpyAsync((uint8_t*)o + vo_off, do_, vo_n, D2H, di->d2h), "copy o")) != LA_OK)
+            return s;
+        if (s_out && (s = cu(cudaMemcpyAsync(s_out + s_off, dso, s_n, D2H, di->d2h), "copy s_out")) != LA_OK)
+            return s;
+        if ((s = cu(cudaEventRecord(ev_out[b], di->d2h), "cudaEventRecord")) != LA_OK) return s;
+    }
+    // the caller's stream continues once the last copy out (and so every one) is done
+    const long last = (U + g - 1) / g - 1;
+    if ((s = cu(cudaStreamWaitEvent(st, ev_out[last & 1], 0), "cudaStreamWaitEvent")) != LA_OK) return s;
+    cleanup();
+    return LA_OK;
 }
 
 la_status la_selftest_wait_timeout(int timeout_us, la_stream_t stream) {

@@ -196,6 +196,30 @@ def test_backward_rejects_bad_arguments(lib, kw, status):
     assert st == status
 
 
+def _host(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, s0=None, s_out=None, B=1, H=4, N=64, dk=128, dv=128, dt=0, group=2,
+             ws=FAKE, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.la_prefill_host(a["q"], a["k"], a["v"], a["o"], a["s0"], a["s_out"], a["B"], a["H"], a["N"],
+                               a["dk"], a["dv"], a["dt"], a["group"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(group=0), 1), (dict(group=-3), 1), (dict(ws=None), 1), (dict(wsb=1000), 1), (dict(ws=FAKE + 8), 1),
+    (dict(q=None), 1), (dict(N=-1), 1), (dict(dk=96, dv=96), 2), (dict(dk=64, dv=128), 2)])
+def test_host_prefill_rejects_bad_arguments(lib, kw, status):
+    assert _host(lib, **kw) == status
+
+
+def test_host_prefill_workspace_size(lib):
+    # two staging buffers, each: q, k, v, o for `group` units and two states
+    g, N, d = 8, 4096, 128
+    per = 4 * g * N * d * 2 + 2 * g * d * d * 4
+    assert lib.la_prefill_host_workspace_size(1, 64, N, d, d, 0, g) == 2 * per
+    assert lib.la_prefill_host_workspace_size(1, 3, N, d, d, 0, g) == 2 * (4 * 3 * N * d * 2 + 2 * 3 * d * d * 4)
+    assert lib.la_prefill_host_workspace_size(1, 64, N, d, d, 0, 0) == 0
+
+
 def test_device_status_null(lib):
     assert lib.la_device_status(None, 0) == 1
 
