@@ -254,7 +254,8 @@ LA_API la_status la_prefill_host(const void* q, const void* k, const void* v, vo
  * bf16 with d = 128: three tensor-core passes of the prefill kernel
  * (dq = prefill(dout, v, k) from s0^T; dk = prefill(v, dout, q) from ds_n^T
  * and dv = prefill(k, q, dout) from ds_n, both with time reversed), with the
- * prefill's precision.  fp32 or d = 64: one FFMA kernel, fp32 arithmetic.
+ * prefill's precision.  fp32 or d = 64: the same three passes on the FFMA
+ * prefill kernel, fp32 arithmetic.
  * d_k = d_v in {64, 128}.  All pointers 16-byte aligned; the caller owns every
  * buffer; no host synchronisation.  Errors: LA_ERR_INVALID_ARG (null, negative,
  * misaligned), LA_ERR_UNSUPPORTED (dims), LA_ERR_CUDA (launch).

@@ -127,7 +127,7 @@ template <> struct Vec<__nv_fp8_e5m2> : VecFp8<__NV_E5M2> {};
 // are half as wide and twice as many units are in flight per SM (measured on
 // B=256, H=64: 5.34 TB/s at 128 threads, 3.34 at 256, 4.46 at 64).
 template <typename SS>
-constexpr int decode_threads() { return Vec<SS>::E == 16 ? NUM_THREADS / 2 : NUM_THREADS; }
+__host__ __device__ constexpr int decode_threads() { return Vec<SS>::E == 16 ? NUM_THREADS / 2 : NUM_THREADS; }
 
 template <typename T, typename SS, int D>
 __global__ void __launch_bounds__(decode_threads<SS>())

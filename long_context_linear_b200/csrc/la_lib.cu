@@ -26,7 +26,6 @@
 #include "selftest.cuh"
 #include "seg_prefix.cuh"
 #include "decode_multi.cuh"
-#include "backward_simt.cuh"
 #include "phi_map.cuh"
 
 namespace lcl {
@@ -252,17 +251,6 @@ void launch_commit(int dk, int m, int grid, const void* k, const void* v, float*
     else launch_commit_d<T, 64>(m, grid, (const T*)k, (const T*)v, S, accepted, H, phi, st);
 }
 
-template <typename T, int D, int CS>
-la_status launch_backward(int grid, const void* q, const void* k, const void* v, const void* dout, void* dq,
-                          void* dk, void* dv, const bwd::Params& bp, cudaStream_t st) {
-    auto kern = bwd::backward_simt_kernel<T, D, CS>;
-    constexpr int smem = bwd::smem_bytes<D, CS>();
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (backward)");
-    kern<<<grid, bwd::NUM_THREADS, smem, st>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, (T*)dq, (T*)dk,
-                                                (T*)dv, bp);
-    return after_launch("backward launch");
-}
 }  // namespace
 }  // namespace lcl
 
@@ -729,7 +717,7 @@ extern "C" la_status la_prefill_varlen_noalloc(const void* q, const void* k, con
 
 // One dense tensor-core pass over whole sequences: o = prefill(q, k, v) from
 // `init` (transposed if init_t), chunks visited last to first if `reverse`.
-la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
+static la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
                         float* s_out, bool reverse, long U, int N, int d, DeviceInfo* di, cudaStream_t st) {
     if (N == 0 && !s_out) return LA_OK;
     tc::Params p{};
@@ -757,6 +745,22 @@ la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, co
     return launch_tc(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_tc (backward pass) launch");
 }
 
+// The same on the FFMA path (fp32 inputs, or d = 64).
+static la_status simt_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
+                          float* s_out, bool reverse, long U, int N, int d, la_dtype dt, cudaStream_t st) {
+    if (N == 0 && !s_out) return LA_OK;
+    simt::Params sp{};
+    sp.mode = 0;
+    sp.N = N;
+    sp.s0 = init;
+    sp.s_out = s_out;
+    sp.phi = LA_PHI_IDENTITY;
+    sp.reverse = reverse ? 1 : 0;
+    sp.init_transposed = init_t ? 1 : 0;
+    if (dt == LA_FP32) return launch_simt<float>(d, 0, (int)U, q, k, v, o, sp, st);
+    return launch_simt<__nv_bfloat16>(d, 0, (int)U, q, k, v, o, sp, st);
+}
+
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,
                               const float* ds_n, void* dq, void* dk, void* dv, float* ds0, int B, int H, int N,
                               int d_k, int d_v, la_dtype dt, la_stream_t stream) {
@@ -775,32 +779,26 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
     DeviceInfo* di;
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // Each gradient is a forward pass over permuted inputs (G_t is the suffix
+    // sum dS_N + sum_{t' >= t} q_t'^T do_t'):
+    //   dq_t = do_t S_t^T : prefill(dO, V, K) from s0^T
+    //   dk_t = v_t G_t^T  : prefill(V, dO, Q) from dS_N^T, chunks last to first
+    //   dv_t = k_t G_t    : prefill(K, Q, dO) from dS_N, chunks last to first;
+    //                       its final state is G_1 = dS_0
+    // on the tensor cores for bf16 with d = 128 (unless LA_BACKWARD_SIMT=1),
+    // else on the FFMA path
     if (use_tensor_cores(d_k, dt) && !env_flag("LA_BACKWARD_SIMT")) {
-        // Each gradient is a forward pass over permuted inputs (G_t is the
-        // suffix sum dS_N + sum_{t' >= t} q_t'^T do_t'):
-        //   dq_t = do_t S_t^T : prefill(dO, V, K) from s0^T
-        //   dk_t = v_t G_t^T  : prefill(V, dO, Q) from dS_N^T, chunks last to first
-        //   dv_t = k_t G_t    : prefill(K, Q, dO) from dS_N, chunks last to first;
-        //                       its final state is G_1 = dS_0
         if (N > 0) {
             if ((s = tc_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, di, st)) != LA_OK) return s;
             if ((s = tc_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, di, st)) != LA_OK) return s;
         }
         return tc_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, di, st);
     }
-    bwd::Params bp{};
-    bp.U = (int)U;
-    bp.N = N;
-    bp.s0 = s0;
-    bp.ds_n = ds_n;
-    bp.ds0 = ds0;
-    const int grid = (int)(2 * U);
-    if (d_k == 128) {
-        if (dt == LA_FP32) return launch_backward<float, 128, 32>(grid, q, k, v, dout, dq, dk, dv, bp, st);
-        return launch_backward<__nv_bfloat16, 128, 32>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+    if (N > 0) {
+        if ((s = simt_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, dt, st)) != LA_OK) return s;
+        if ((s = simt_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, dt, st)) != LA_OK) return s;
     }
-    if (dt == LA_FP32) return launch_backward<float, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
-    return launch_backward<__nv_bfloat16, 64, 64>(grid, q, k, v, dout, dq, dk, dv, bp, st);
+    return simt_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, dt, st);
 }
 
 size_t la_prefill_host_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt, int group) {

@@ -8,8 +8,13 @@
 //   A   = (Q_c K_c^T) ⊙ M        M keeps s <= t
 //   O_c = A V_c + Q_c S
 //   S  += K_c^T V_c
-// One CTA per (unit | sequence, head); the whole d x d fp32 state lives in
-// shared memory.  The chunk length CS (32 or 64) is a template parameter.
+// One CTA per (unit | sequence, head), 256 threads.  Every product is
+// register-tiled (each thread owns a block of outputs and reads 16-byte
+// vectors from shared memory), tiles wholly above the causal diagonal are
+// skipped, the state S stays in the registers of its owner threads between
+// chunks (and in shared memory for Q S), and the next chunk is prefetched into
+// L2 while this one is loaded.  The chunk length CS (32 or 64) is a template
+// parameter.
 #pragma once
 #include "phi.cuh"
 #include <cuda_bf16.h>
@@ -29,6 +34,10 @@ struct Params {
     const int* init_idx;    // packed: [n_seq] or null
     float* s_out;           // [U | n_seq*H][d][d] or null
     int phi;                // feature map applied to q and k (phi.cuh)
+    // dense only: visit the chunks last to first and keep s >= t inside a
+    // chunk, so that o_t = q_t (S_init + sum_{s >= t} k_s v_s^T)
+    int reverse;
+    int init_transposed;    // the initial state is given as its transpose [d][d]
 };
 
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -37,23 +46,124 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Shared-memory layout (floats), rows padded by 4 so that 16-byte vectors
+// stay aligned and successive rows start in different banks:
+//   Qt, Kt [D][CS+4]   Q and K transposed (token index contiguous)
+//   Vn     [CS][D+4]   V as stored
+//   At     [CS][CS+4]  masked scores, transposed: At[s][t] = (q_t . k_s) [s <= t]
+//   Sm     [D][D+4]    the state before this chunk
 template <int D, int CS>
 constexpr int smem_bytes() {
-    return (D * D + 3 * CS * (D + 1) + CS * (CS + 1)) * 4;
+    return (2 * D * (CS + 4) + CS * (D + 4) + CS * (CS + 4) + D * (D + 4)) * 4;
 }
 
+// Register tiles: the 256 threads form a 16 x 16 grid (ty = tid / 16 picks
+// the tile row, tx = tid % 16 the tile column); each thread owns TM x TN
+// outputs of a product.  Tile rows are a contiguous block (ty*TM ...); tile
+// columns come in groups of 4 spread N / (TN/4) apart (tx*4 ... within each
+// group), so that the 16 threads of a row read one contiguous stretch per
+// 16-byte load.
+template <int TN, int N>
+__device__ __forceinline__ int col_of(int tx, int c) {
+    if constexpr (TN >= 4) return (c / 4) * (N / (TN / 4)) + tx * 4 + (c % 4);
+    else return tx * TN + c;
+}
+
+// TN values of one row for thread column tx
+template <int TN, int N>
+__device__ __forceinline__ void ld_cols(const float* row, int tx, float (&x)[TN]) {
+    if constexpr (TN >= 4) {
+#pragma unroll
+        for (int g = 0; g < TN / 4; ++g) {
+            const float4 v = *reinterpret_cast<const float4*>(row + g * (N / (TN / 4)) + tx * 4);
+            x[4 * g] = v.x; x[4 * g + 1] = v.y; x[4 * g + 2] = v.z; x[4 * g + 3] = v.w;
+        }
+    } else {
+        const float2 v = *reinterpret_cast<const float2*>(row + tx * 2);
+        x[0] = v.x; x[1] = v.y;
+    }
+}
+template <int TN, int N>
+__device__ __forceinline__ void st_cols(float* row, int tx, const float (&x)[TN]) {
+    if constexpr (TN >= 4) {
+#pragma unroll
+        for (int g = 0; g < TN / 4; ++g)
+            *reinterpret_cast<float4*>(row + g * (N / (TN / 4)) + tx * 4) =
+                make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+    } else {
+        *reinterpret_cast<float2*>(row + tx * 2) = make_float2(x[0], x[1]);
+    }
+}
+// TM contiguous values (TM = 2, 4 or 8) at p, 8-byte aligned at least
+template <int TM>
+__device__ __forceinline__ void ld_run(const float* p, float (&x)[TM]) {
+    if constexpr (TM % 4 == 0) {
+#pragma unroll
+        for (int g = 0; g < TM / 4; ++g) {
+            const float4 v = *reinterpret_cast<const float4*>(p + 4 * g);
+            x[4 * g] = v.x; x[4 * g + 1] = v.y; x[4 * g + 2] = v.z; x[4 * g + 3] = v.w;
+        }
+    } else {
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        x[0] = v.x; x[1] = v.y;
+    }
+}
+template <int TM>
+__device__ __forceinline__ void st_run(float* p, const float (&x)[TM]) {
+    if constexpr (TM % 4 == 0) {
+#pragma unroll
+        for (int g = 0; g < TM / 4; ++g)
+            *reinterpret_cast<float4*>(p + 4 * g) = make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+    } else {
+        *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+    }
+}
+
+// 16 bytes of T -> fp32
+__device__ __forceinline__ void unpack16(const uint4 r, float (&f)[4]) {
+    f[0] = __uint_as_float(r.x); f[1] = __uint_as_float(r.y); f[2] = __uint_as_float(r.z); f[3] = __uint_as_float(r.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 r, float (&f)[8]) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+// 4 outputs -> T at p (16 bytes for fp32, 8 for bf16)
+__device__ __forceinline__ void store4(float* p, const float* x) { *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]); }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float* x) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+    *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
+__device__ __forceinline__ void store2(float* p, const float* x) { *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]); }
+__device__ __forceinline__ void store2(__nv_bfloat16* p, const float* x) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
+    *reinterpret_cast<uint32_t*>(p) = *reinterpret_cast<const uint32_t*>(&a);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 template <typename T, int D, int CS>
-__global__ void __launch_bounds__(NUM_THREADS)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
 prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
                     const Params p) {
+    static_assert(CS == 32 || CS == 64, "chunk of 32 or 64 tokens");
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    constexpr int LQ = CS + 4, LV = D + 4;
+    constexpr int TM1 = CS / 16, TN1 = CS / 16;   // scores   [CS x CS]
+    constexpr int TM2 = CS / 16, TN2 = D / 16;    // outputs  [CS x D]
+    constexpr int TM3 = D / 16, TN3 = D / 16;     // state    [D x D]
+    constexpr int VEC = 16 / sizeof(T);           // elements per 16-byte global load
+    constexpr int VPR = D / VEC;                  // 16-byte vectors per row
     extern __shared__ float sf[];
-    float* S = sf;                   // [D][D]
-    float* Qs = S + D * D;           // [CS][D+1]
-    float* Ks = Qs + CS * (D + 1);
-    float* Vs = Ks + CS * (D + 1);
-    float* A = Vs + CS * (D + 1);    // [CS][CS+1]
-    constexpr int LD = D + 1;
-    const int tid = threadIdx.x;
+    float* Qt = sf;
+    float* Kt = Qt + D * LQ;
+    float* Vn = Kt + D * LQ;
+    float* At = Vn + CS * LV;
+    float* Sm = At + CS * LQ;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
 
     long row0, row_stride, state;
     int len;
@@ -75,57 +185,158 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         const int ii = p.init_idx ? p.init_idx[seq] : -1;
         if (p.pool && ii >= 0) init = p.pool + ((long)ii * p.H + h) * D * D;
     }
-    for (int e = tid; e < D * D; e += NUM_THREADS) S[e] = init ? init[e] : 0.f;
-
-    for (int c0 = 0; c0 < len; c0 += CS) {
-        const int rows = min(CS, len - c0);
-        __syncthreads();
-        for (int e = tid; e < CS * D; e += NUM_THREADS) {
-            const int t = e / D, i = e % D;
-            float a = 0.f, b = 0.f, cc = 0.f;
-            if (t < rows) {
-                const long g = (row0 + (long)(c0 + t) * row_stride) * D + i;
-                a = apply_phi(to_f(q[g]), p.phi);
-                b = apply_phi(to_f(k[g]), p.phi);
-                cc = to_f(v[g]);
-            }
-            Qs[t * LD + i] = a;
-            Ks[t * LD + i] = b;
-            Vs[t * LD + i] = cc;
+    // the state tile of this thread: rows ty*TM3 + r, columns col_of<TN3, D>(tx, c)
+    float accS[TM3][TN3];
+#pragma unroll
+    for (int r = 0; r < TM3; ++r) {
+        const int i = ty * TM3 + r;
+#pragma unroll
+        for (int c = 0; c < TN3; ++c) {
+            const int j = col_of<TN3, D>(tx, c);
+            accS[r][c] = init ? init[p.init_transposed ? j * D + i : i * D + j] : 0.f;
         }
-        __syncthreads();
-        for (int e = tid; e < CS * CS; e += NUM_THREADS) {
-            const int t = e / CS, s = e % CS;
-            float a = 0.f;
-            if (s <= t) {
-#pragma unroll 8
-                for (int i = 0; i < D; ++i) a = fmaf(Qs[t * LD + i], Ks[s * LD + i], a);
-            }
-            A[t * (CS + 1) + s] = a;
-        }
-        __syncthreads();
-        for (int e = tid; e < CS * D; e += NUM_THREADS) {
-            const int t = e / D, j = e % D;
-            if (t < rows) {
-                float acc = 0.f;
-                for (int s = 0; s <= t; ++s) acc = fmaf(A[t * (CS + 1) + s], Vs[s * LD + j], acc);
-#pragma unroll 8
-                for (int i = 0; i < D; ++i) acc = fmaf(Qs[t * LD + i], S[i * D + j], acc);
-                o[(row0 + (long)(c0 + t) * row_stride) * D + j] = from_f<T>(acc);
-            }
-        }
-        __syncthreads();
-        for (int e = tid; e < D * D; e += NUM_THREADS) {
-            const int i = e / D, j = e % D;
-            float acc = S[e];
-            for (int s = 0; s < rows; ++s) acc = fmaf(Ks[s * LD + i], Vs[s * LD + j], acc);
-            S[e] = acc;
-        }
+        st_cols<TN3, D>(Sm + i * LV, tx, accS[r]);
     }
-    __syncthreads();
+
+    const bool rev = p.reverse;
+    const int nc = (len + CS - 1) / CS;
+    for (int ci = 0; ci < nc; ++ci) {
+        const int c0 = (rev ? nc - 1 - ci : ci) * CS;
+        const int rows = min(CS, len - c0);
+        __syncthreads();  // the previous chunk is done with Qt, Kt, Vn, At and Sm
+        // ---- next chunk into L2, this chunk into shared memory (phi on q and k)
+        if (ci + 1 < nc) {
+            constexpr int LINES = D * (int)sizeof(T) / 128;
+            const int n0 = (rev ? nc - 2 - ci : ci + 1) * CS;
+            const int nrows = min(CS, len - n0);
+            for (int f = tid; f < 3 * nrows * LINES; f += NUM_THREADS) {
+                const int which = f / (nrows * LINES), rl = f % (nrows * LINES);
+                const long g = (row0 + (long)(n0 + rl / LINES) * row_stride) * D;
+                const T* src = which == 0 ? q : (which == 1 ? k : v);
+                prefetch_l2(src + g + (rl % LINES) * (128 / (int)sizeof(T)));
+            }
+        }
+        for (int f = tid; f < CS * VPR; f += NUM_THREADS) {
+            const int t = f / VPR, cc = (f % VPR) * VEC;
+            float qv[VEC], kv[VEC], vv[VEC];
+            if (t < rows) {
+                const long g = (row0 + (long)(c0 + t) * row_stride) * D + cc;
+                unpack16(*reinterpret_cast<const uint4*>(q + g), qv);
+                unpack16(*reinterpret_cast<const uint4*>(k + g), kv);
+                unpack16(*reinterpret_cast<const uint4*>(v + g), vv);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    qv[e] = apply_phi(qv[e], p.phi);
+                    kv[e] = apply_phi(kv[e], p.phi);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) qv[e] = kv[e] = vv[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                Qt[(cc + e) * LQ + t] = qv[e];
+                Kt[(cc + e) * LQ + t] = kv[e];
+            }
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4*>(Vn + t * LV + cc + e) = make_float4(vv[e], vv[e + 1], vv[e + 2], vv[e + 3]);
+        }
+        __syncthreads();
+        // ---- scores: At[s][t] = q_t . k_s for s <= t (s >= t in reverse), else 0
+        {
+            const int t0 = ty * TM1, s0 = tx * TN1;
+            float acc[TM1][TN1];
+#pragma unroll
+            for (int r = 0; r < TM1; ++r)
+#pragma unroll
+                for (int c = 0; c < TN1; ++c) acc[r][c] = 0.f;
+            if (rev ? s0 + TN1 - 1 >= t0 : s0 <= t0 + TM1 - 1) {  // the tile holds kept entries
+#pragma unroll 4
+                for (int i = 0; i < D; ++i) {
+                    float a[TM1], b[TN1];
+                    ld_run<TM1>(Qt + i * LQ + t0, a);
+                    ld_run<TN1>(Kt + i * LQ + s0, b);
+#pragma unroll
+                    for (int r = 0; r < TM1; ++r)
+#pragma unroll
+                        for (int c = 0; c < TN1; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < TN1; ++c) {
+                float col[TM1];
+#pragma unroll
+                for (int r = 0; r < TM1; ++r) col[r] = (rev ? s0 + c >= t0 + r : s0 + c <= t0 + r) ? acc[r][c] : 0.f;
+                st_run<TM1>(At + (s0 + c) * LQ + t0, col);
+            }
+        }
+        __syncthreads();
+        // ---- outputs: O_t = sum_s At[s][t] v_s + q_t S (s <= t, or s >= t in reverse)
+        {
+            const int t0 = ty * TM2;
+            float acc[TM2][TN2];
+#pragma unroll
+            for (int r = 0; r < TM2; ++r)
+#pragma unroll
+                for (int c = 0; c < TN2; ++c) acc[r][c] = 0.f;
+            const int smin = rev ? t0 : 0, smax = rev ? rows : min(rows, t0 + TM2);
+#pragma unroll 2
+            for (int s = smin; s < smax; ++s) {
+                float a[TM2], b[TN2];
+                ld_run<TM2>(At + s * LQ + t0, a);
+                ld_cols<TN2, D>(Vn + s * LV, tx, b);
+#pragma unroll
+                for (int r = 0; r < TM2; ++r)
+#pragma unroll
+                    for (int c = 0; c < TN2; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+            }
+#pragma unroll 4
+            for (int i = 0; i < D; ++i) {
+                float a[TM2], b[TN2];
+                ld_run<TM2>(Qt + i * LQ + t0, a);
+                ld_cols<TN2, D>(Sm + i * LV, tx, b);
+#pragma unroll
+                for (int r = 0; r < TM2; ++r)
+#pragma unroll
+                    for (int c = 0; c < TN2; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+            }
+#pragma unroll
+            for (int r = 0; r < TM2; ++r) {
+                if (t0 + r >= rows) break;
+                T* dst = o + (row0 + (long)(c0 + t0 + r) * row_stride) * D;
+                if constexpr (TN2 >= 4) {
+#pragma unroll
+                    for (int g = 0; g < TN2 / 4; ++g) store4(dst + col_of<TN2, D>(tx, 4 * g), &acc[r][4 * g]);
+                } else {
+                    store2(dst + col_of<TN2, D>(tx, 0), &acc[r][0]);
+                }
+            }
+        }
+        __syncthreads();  // every read of Sm for this chunk is done
+        // ---- state: S += K^T V over the chunk's valid rows
+#pragma unroll 2
+        for (int s = 0; s < rows; ++s) {
+            float a[TM3], b[TN3];
+#pragma unroll
+            for (int r = 0; r < TM3; ++r) a[r] = Kt[(ty * TM3 + r) * LQ + s];
+            ld_cols<TN3, D>(Vn + s * LV, tx, b);
+#pragma unroll
+            for (int r = 0; r < TM3; ++r)
+#pragma unroll
+                for (int c = 0; c < TN3; ++c) accS[r][c] = fmaf(a[r], b[c], accS[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < TM3; ++r) st_cols<TN3, D>(Sm + (ty * TM3 + r) * LV, tx, accS[r]);
+    }
     if (p.s_out) {
         float* dst = p.s_out + state * D * D;
-        for (int e = tid; e < D * D; e += NUM_THREADS) dst[e] = S[e];
+#pragma unroll
+        for (int r = 0; r < TM3; ++r) {
+            const int i = ty * TM3 + r;
+#pragma unroll
+            for (int c = 0; c < TN3; ++c) dst[i * D + col_of<TN3, D>(tx, c)] = accS[r][c];
+        }
     }
 }
 

@@ -100,3 +100,19 @@ def test_backward_tc_no_ds0(la, oracle_mod):
     rq, rk, rv, _ = oracle_mod.backward(q, k, v, dout)
     for g, r in ((dq, rq), (dk, rk), (dv, rv)):
         assert_out(g.cpu(), r, torch.bfloat16, 2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_ffma_integer_inputs_bit_exact(la, oracle_mod, d):
+    """fp32 inputs in {-1,0,1} with integer states: the FFMA passes keep every
+    product and partial sum exact, so all four gradients equal the oracle's bit
+    for bit."""
+    B, H, N = 1, 2, 300
+    q, k, v, dout = (synth.integer_valued((B, H, N, d), seed=s) for s in (21, 22, 23, 24))
+    s0 = synth.integer_valued((B, H, d, d), seed=25, lo=-20, hi=20)
+    ds_n = synth.integer_valued((B, H, d, d), seed=26, lo=-20, hi=20)
+    dq, dk, dv, ds0 = la.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), s0.cuda(), ds_n.cuda())
+    torch.cuda.synchronize()
+    rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
+    for g, r in ((dq, rq), (dk, rk), (dv, rv), (ds0, rs0)):
+        np.testing.assert_array_equal(to64(g.cpu()), r)
