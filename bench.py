@@ -453,9 +453,36 @@ def run_backward(args, dist: Dist, pk):
     gbs = byts / (ms_step / 1e3) / 1e9
     del q, k, v, do
     torch.cuda.empty_cache()
-    return dict(workload="backward of prefill B=4 H=32 N=8192 d=128 bf16 (three tensor-core passes)",
-                tokens_per_s=B * N * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
-                frac=gbs / pk["hbm"], steps=n)
+    res = dict(workload="backward of prefill B=4 H=32 N=8192 d=128 bf16 (three tensor-core passes)",
+               tokens_per_s=B * N * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
+               frac=gbs / pk["hbm"], steps=n)
+    # few heads, long sequence: the passes cut into segments, and unsplit
+    c = FEWHEADS
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=83 + dist.rank, device=dev)
+    _, _, do = synth.dense(B, H, N, d, "bf16", seed=93 + dist.rank, device=dev)
+    ws = torch.empty(max(la.lib.la_prefill_backward_workspace_size(B, H, N, d, d, 0), 1), dtype=torch.uint8,
+                     device=dev)
+    few = dict(workload="backward of prefill B=1 H=8 N=131072 d=128 bf16", workspace_bytes=ws.numel())
+    prev = os.environ.get("LA_PREFILL_SEGMENTS")
+    try:
+        for key, env in (("split", None), ("unsplit", "1")):
+            if env is None:
+                os.environ.pop("LA_PREFILL_SEGMENTS", None)
+            else:
+                os.environ["LA_PREFILL_SEGMENTS"] = env
+            total_ms, _ = timed_launches(lambda: la.prefill_backward(q, k, v, do, workspace=ws), n,
+                                         max(3, args.warmup), dist, stream)
+            few[key] = dict(ms_per_step=dist.max(total_ms) / n)
+    finally:
+        if prev is None:
+            os.environ.pop("LA_PREFILL_SEGMENTS", None)
+        else:
+            os.environ["LA_PREFILL_SEGMENTS"] = prev
+    res["few_heads"] = few
+    del q, k, v, do, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_few_heads(args, dist: Dist, pk):

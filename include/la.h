@@ -265,6 +265,16 @@ LA_API la_status la_prefill_backward(const void* q, const void* k, const void* v
                                      void* dq, void* dk, void* dv, float* ds0,
                                      int B, int H, int N, int d_k, int d_v, la_dtype dt,
                                      la_stream_t stream);
+/* la_prefill_backward with a workspace (device, 16-byte aligned) of at least
+ * la_prefill_backward_workspace_size(...) bytes: when the (batch, head) units
+ * fill less than half of the SMs, each tensor-core pass cuts the sequences
+ * into segments as la_prefill does (in reverse order the segment starts are
+ * suffix sums).  With a smaller workspace (or none) the passes run unsplit. */
+LA_API size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v, la_dtype dt);
+LA_API la_status la_prefill_backward_ex(const void* q, const void* k, const void* v, const void* dout,
+                                        const float* s0, const float* ds_n, void* dq, void* dk, void* dv, float* ds0,
+                                        int B, int H, int N, int d_k, int d_v, la_dtype dt, void* workspace,
+                                        size_t ws_bytes, la_stream_t stream);
 
 /*
  * Reads the device status word of the current device (synchronizes the

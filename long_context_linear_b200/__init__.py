@@ -161,7 +161,7 @@ def prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s0: Optional
 
 def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,
                      s0: Optional[torch.Tensor] = None, ds_n: Optional[torch.Tensor] = None, *,
-                     need_ds0: bool = True):
+                     need_ds0: bool = True, workspace: Optional[torch.Tensor] = None):
     """Gradients of ``prefill`` for dL/dO = dout and dL/dS_N = ds_n (zero if None).
 
     q, k, v, dout: [B, H, N, d]; s0, ds_n: fp32 [B, H, d, d] or None.
@@ -180,10 +180,14 @@ def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: to
                 raise ValueError(f"{n} must be [B, H, d, d]")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ds0 = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if need_ds0 else None
+    need = int(lib.la_prefill_backward_workspace_size(B, H, N, d, d, _dtype_code(q)))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
-        _abi.check(lib.la_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(s0), _ptr(ds_n), _ptr(dq),
-                                           _ptr(dk), _ptr(dv), _ptr(ds0), B, H, N, d, d, _dtype_code(q),
-                                           _stream(q.device)), "la_prefill_backward")
+        _abi.check(lib.la_prefill_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(s0), _ptr(ds_n), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), _ptr(ds0), B, H, N, d, d, _dtype_code(q),
+                                              _ptr(workspace), ws_bytes, _stream(q.device)), "la_prefill_backward_ex")
     return dq, dk, dv, ds0
 
 

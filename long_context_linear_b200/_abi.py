@@ -52,6 +52,9 @@ SIGNATURES = {
     "la_prefill_host_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "la_prefill_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "la_prefill_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "la_prefill_backward_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "la_prefill_backward_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz,
+                                    _vp]),
     "la_device_status": (_i, [ctypes.POINTER(_i), _i]),
     "la_selftest_wait_timeout": (_i, [_i, _vp]),
     "la_prefill_varlen_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),

@@ -444,7 +444,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
             return s;
         const long threads = U * (long)(dk * dv / 4);
         const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
-        segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(seg_sums, s0, starts, U, P, dk * dv);
+        segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(seg_sums, s0, starts, U, P, dk * dv, 0, 0, dk);
         if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
         p.n_seg = P;
         p.n_items = (int)(U * P * tc::NVS);
@@ -715,10 +715,14 @@ extern "C" la_status la_prefill_varlen_noalloc(const void* q, const void* k, con
                              chunk, scratch, sizeof(int) * LA_NOALLOC_MAX_SEQS, stream);
 }
 
-// One dense tensor-core pass over whole sequences: o = prefill(q, k, v) from
-// `init` (transposed if init_t), chunks visited last to first if `reverse`.
+// One dense tensor-core pass: o = prefill(q, k, v) from `init` (transposed if
+// init_t), chunks visited last to first if `reverse`.  When the (unit, value
+// slice) items fill less than half of the SMs and `ws` has room, sequences are
+// cut into segments as in la_prefill_ex (a state-only pass, then a prefix --
+// in reverse order a suffix -- over the segment sums, then every segment).
 static la_status tc_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
-                        float* s_out, bool reverse, long U, int N, int d, DeviceInfo* di, cudaStream_t st) {
+                               float* s_out, bool reverse, long U, int N, int d, DeviceInfo* di, cudaStream_t st,
+                               void* ws, size_t ws_bytes) {
     if (N == 0 && !s_out) return LA_OK;
     tc::Params p{};
     p.mode = 0;
@@ -730,10 +734,15 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.status = di->status;
     p.n_seg = 1;
-    p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
     p.phi = LA_PHI_IDENTITY;
     p.reverse = reverse ? 1 : 0;
     p.init_transposed = init_t ? 1 : 0;
+    int seg_len;
+    int P = plan_segments(U, N, di->sms, &seg_len);
+    if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) ||
+                  U * P * tc::NVS > (1L << 30)))
+        P = 1;
+    p.seg_len = P > 1 ? seg_len : ((N + tc::C - 1) / tc::C) * tc::C;
     const void* any = N > 0 ? q : s_out;
     CUtensorMap mq, mk, mv, mo;
     const uint64_t row = (uint64_t)d * 2, Nm = N > 0 ? (uint64_t)N : 1, unit = Nm * row;
@@ -742,6 +751,31 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     if ((s = make_map(&mk, N > 0 ? k : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mv, N > 0 ? v : any, d, Nm, U, row, unit, tc::C, 1)) != LA_OK) return s;
     if ((s = make_map(&mo, N > 0 ? o : any, d, Nm, U, row, unit, 32, 1)) != LA_OK) return s;
+    if (P > 1) {
+        float* sums = reinterpret_cast<float*>(ws);
+        float* starts = sums + (size_t)U * (P - 1) * d * d;
+        tc::Params p1 = p;
+        p1.n_seg = P - 1;
+        p1.seg_base = reverse ? 1 : 0;  // the segments whose sums reach another segment's start
+        p1.n_items = (int)(U * (P - 1) * tc::NVS);
+        p1.s0 = nullptr;
+        p1.init_transposed = 0;
+        p1.s_out = sums;
+        p1.s_out_per_seg = 1;
+        p1.state_only = 1;
+        if ((s = launch_tc(std::min(p1.n_items, di->sms), mq, mk, mv, mo, p1, st, "prefill_tc (segment sums) launch")) !=
+            LA_OK)
+            return s;
+        const long threads = U * (long)(d * d / 4);
+        const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
+        segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(sums, init, starts, U, P, d * d, reverse ? 1 : 0,
+                                                                     init_t ? 1 : 0, d);
+        if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
+        p.n_seg = P;
+        p.n_items = (int)(U * P * tc::NVS);
+        p.seg_init = starts;
+        p.init_transposed = 0;  // the segment starts are in the usual layout
+    }
     return launch_tc(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_tc (backward pass) launch");
 }
 
@@ -761,9 +795,26 @@ static la_status simt_dense_pass(const void* q, const void* k, const void* v, vo
     return launch_simt<__nv_bfloat16>(d, 0, (int)U, q, k, v, o, sp, st);
 }
 
+size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v, la_dtype dt) {
+    if (B <= 0 || H <= 0 || N <= 0 || !use_tensor_cores(d_k, dt) || d_k != d_v) return 0;
+    DeviceInfo* di;
+    if (device_info(&di) != LA_OK) return 0;
+    int seg_len;
+    const long U = (long)B * H;
+    return segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), d_k, d_v);
+}
+
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,
                               const float* ds_n, void* dq, void* dk, void* dv, float* ds0, int B, int H, int N,
                               int d_k, int d_v, la_dtype dt, la_stream_t stream) {
+    return la_prefill_backward_ex(q, k, v, dout, s0, ds_n, dq, dk, dv, ds0, B, H, N, d_k, d_v, dt, nullptr, 0,
+                                  stream);
+}
+
+la_status la_prefill_backward_ex(const void* q, const void* k, const void* v, const void* dout, const float* s0,
+                                 const float* ds_n, void* dq, void* dk, void* dv, float* ds0, int B, int H, int N,
+                                 int d_k, int d_v, la_dtype dt, void* workspace, size_t ws_bytes,
+                                 la_stream_t stream) {
     g_last_error[0] = 0;
     la_status s = check_dims(d_k, d_v, dt);
     if (s != LA_OK) return s;
@@ -789,10 +840,15 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
     // else on the FFMA path
     if (use_tensor_cores(d_k, dt) && !env_flag("LA_BACKWARD_SIMT")) {
         if (N > 0) {
-            if ((s = tc_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, di, st)) != LA_OK) return s;
-            if ((s = tc_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, di, st)) != LA_OK) return s;
+            if ((s = tc_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, di, st, workspace, ws_bytes)) !=
+                LA_OK)
+                return s;
+            if ((s = tc_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, di, st, workspace, ws_bytes)) !=
+                LA_OK)
+                return s;
         }
-        return tc_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, di, st);
+        // (the passes run in stream order, so they share the workspace)
+        return tc_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, di, st, workspace, ws_bytes);
     }
     if (N > 0) {
         if ((s = simt_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, dt, st)) != LA_OK) return s;

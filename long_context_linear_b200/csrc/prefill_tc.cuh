@@ -117,6 +117,7 @@ struct Params {
     // inside a chunk, so that o_t = q_t (S_init + sum_{s >= t} k_s v_s^T)
     int reverse;
     int init_transposed;   // the initial state is given as its transpose [dv][DK]
+    int seg_base;          // dense: the items' segments are seg_base .. seg_base + n_seg - 1
 };
 
 struct Item {
@@ -155,14 +156,16 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     } else if (p.mode == 0) {
         const int us = idx / NVS;  // unit * n_seg + segment
         const int u = us / p.n_seg, sg = us - u * p.n_seg;
-        it.t0 = sg * p.seg_len;
+        // the segment visited first starts from s0; the one visited last ends the sequence
+        const int first = p.reverse ? p.n_seg - 1 : 0, last = p.reverse ? 0 : p.n_seg - 1;
+        it.t0 = (sg + p.seg_base) * p.seg_len;
         it.len = min(p.seg_len, p.N - it.t0);
         it.c1 = 0;
         it.c2 = u;
         it.state = p.s_out_per_seg ? us : u;
         it.init = p.seg_init ? p.seg_init + (long)us * DK * p.dv
-                             : ((sg == 0 && p.s0) ? p.s0 + (long)u * DK * p.dv : nullptr);
-        it.write_state = p.s_out_per_seg || sg == p.n_seg - 1;
+                             : ((sg == first && p.s0) ? p.s0 + (long)u * DK * p.dv : nullptr);
+        it.write_state = p.s_out_per_seg || sg == last;
     } else {
         const int hs = idx / NVS;   // sequence rank * H + head
         const int r = hs / p.H;

@@ -116,3 +116,36 @@ def test_backward_ffma_integer_inputs_bit_exact(la, oracle_mod, d):
     rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
     for g, r in ((dq, rq), (dk, rk), (dv, rv), (ds0, rs0)):
         np.testing.assert_array_equal(to64(g.cpu()), r)
+
+
+@pytest.mark.parametrize("segments", ["2", "3", "5"])
+def test_backward_tc_segments_match_oracle(la, oracle_mod, monkeypatch, segments):
+    """Each tensor-core pass cut into segments (state-only pass, prefix or, in
+    reverse order, suffix over the segment sums, then all segments)."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v, dout, s0, ds_n = _grad_case(1, 2, 3000, 128, "bf16", seed=31, with_states=True)
+    dq, dk, dv, ds0 = la.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), s0.cuda(), ds_n.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
+    for g, r in ((dq, rq), (dk, rk), (dv, rv)):
+        assert_out(g.cpu(), r, torch.bfloat16, 2)
+    assert_state(ds0.cpu(), rs0, 2, tol=1e-4)
+
+
+@pytest.mark.parametrize("segments", ["1", "4"])
+def test_backward_tc_segments_integer_inputs_bit_exact(la, oracle_mod, monkeypatch, segments):
+    """With inputs in {-1,0,1} every sum is exact whatever its order, so the
+    segmented passes equal the oracle bit for bit, like the unsplit ones."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N, d = 1, 2, 1500, 128
+    q, k, v, dout = (synth.integer_valued((B, H, N, d), seed=s, dtype=torch.bfloat16) for s in (41, 42, 43, 44))
+    s0 = synth.integer_valued((B, H, d, d), seed=45, lo=-20, hi=20, dtype=torch.float32)
+    ds_n = synth.integer_valued((B, H, d, d), seed=46, lo=-20, hi=20, dtype=torch.float32)
+    dq, dk, dv, ds0 = la.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), s0.cuda(), ds_n.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
+    for g, r in ((dq, rq), (dk, rk), (dv, rv)):
+        assert torch.equal(g.cpu(), torch.from_numpy(r).to(torch.bfloat16))
+    np.testing.assert_array_equal(to64(ds0.cpu()), rs0)
