@@ -99,3 +99,17 @@ def test_varlen_validation_rejects_bad_offsets(la, monkeypatch):
         la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), pool.cuda(), bad_idx.cuda())
     o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), pool.cuda(), idx.cuda())
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("n_seq", [4096, 5000])
+def test_varlen_many_short_sequences(la, oracle_mod, n_seq):
+    """The largest batch the device sort orders longest-first (4096), and one
+    beyond it (kept in its own order); lengths 0 .. 24, a third resumed."""
+    rng = np.random.default_rng(n_seq)
+    lens = [int(x) for x in rng.integers(0, 25, n_seq)]
+    resume = [int(x) for x in rng.integers(-1, 3, n_seq)]
+    cu, q, k, v, pool, idx = _case(lens, 2, 128, "bf16", seed=9, n_pool=3, resume=resume)
+    o, s = _run(la, cu, q, k, v, pool, idx)
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_state(s, rs, 2)
