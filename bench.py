@@ -317,6 +317,45 @@ def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
                 bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
 
 
+def run_decode_small_graph(args, dist: Dist, pk):
+    """Decode at a small batch (B=4, H=64: 16 MiB of state per step), where a
+    step is launch-bound: 1024 eager calls against the same 1024 steps
+    captured once in a CUDA graph and replayed."""
+    import long_context_linear_b200 as la
+    import synth
+    B, H, d, steps = 4, 64, 128, 1024
+    dev = torch.device("cuda", torch.cuda.current_device())
+    S0 = synth.outer_product_state(B * H, d, d, [4096] * (B * H), seed=45 + dist.rank, device=dev).view(B, H, d, d)
+    qs, ks, vs = synth.qkv((steps, B, H, d), d, "bf16", seed=47 + dist.rank, device=dev)
+    os_ = torch.empty_like(vs)
+    S = S0.clone()
+    stream = torch.cuda.current_stream(dev)
+
+    def eager():
+        for t in range(steps):
+            la.decode_step(qs[t], ks[t], vs[t], S, out=os_[t])
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        eager()
+    stream.wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        eager()
+    n = 3
+    e_ms, _ = timed_launches(eager, n, max(3, args.warmup), dist, stream)
+    g_ms, _ = timed_launches(g.replay, n, max(3, args.warmup), dist, stream)
+    e_step, g_step = dist.max(e_ms) / (n * steps), dist.max(g_ms) / (n * steps)
+    byts = 2.0 * B * H * d * d * 4 + 4.0 * B * H * d * 2
+    del g, S, S0, qs, ks, vs, os_
+    torch.cuda.empty_cache()
+    return dict(workload="decode B=4 H=64 d=128, fp32 state, 1024 steps", eager_us_per_step=e_step * 1e3,
+                graph_us_per_step=g_step * 1e3, tokens_per_s_eager=B * dist.world / (e_step / 1e3),
+                tokens_per_s_graph=B * dist.world / (g_step / 1e3), hbm_gbs_graph=byts / (g_step / 1e3) / 1e9,
+                frac_graph=byts / (g_step / 1e3) / 1e9 / pk["hbm"])
+
+
 def run_speculative(args, dist: Dist, pk, m: int = 4):
     """Decode B=256, H=64 with m draft tokens per step: one verify and one
     commit of all m drafts, against m plain decode steps (same states)."""
@@ -618,6 +657,7 @@ def main():
         extras["decode_bf16_state"] = run_decode(args, dist, pk, torch.bfloat16)
         extras["decode_fp16_state"] = run_decode(args, dist, pk, torch.float16)
         extras["decode_fp8_e4m3_state"] = run_decode(args, dist, pk, torch.float8_e4m3fn)
+        extras["decode_small_graph"] = run_decode_small_graph(args, dist, pk)
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
