@@ -153,3 +153,19 @@ def test_unsupported_chunk_raises(la):
     q, k, v = synth.dense(1, 1, 10, 128, "bf16", seed=0)
     with pytest.raises(la.LAError):
         la.prefill(q.cuda(), k.cuda(), v.cuda(), chunk=48)
+
+
+def test_tc_many_units_per_cta(la, oracle_mod):
+    """512 (batch, head) units = 1024 items on the persistent grid (about 7
+    items per CTA, boustrophedon order), each with a ragged last chunk and its
+    own initial state; a sample of units against the oracle."""
+    B, H, N = 32, 16, 200
+    q, k, v = synth.dense(B, H, N, 128, "bf16", seed=71)
+    s0 = _state(B, H, 128, seed=72, L=100)
+    o, s = _run(la, q, k, v, s0)
+    units = synth.choose(B * H, 24, seed=73)
+    qf, kf, vf, of, sf, s0f = (x.reshape(B * H, *x.shape[2:]) for x in (q, k, v, o, s, s0))
+    idx = torch.tensor(units)
+    ro, rs = oracle_mod.recurrent(qf[idx], kf[idx], vf[idx], s0f[idx])
+    assert_out(of[idx], ro, torch.bfloat16, 1)
+    assert_state(sf[idx], rs, 1)
