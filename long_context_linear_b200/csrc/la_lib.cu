@@ -104,11 +104,14 @@ la_status device_info(DeviceInfo** out) {
             return cuda_fail(e, "cudaDeviceGetAttribute");
         if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word)) != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress");
-        if ((e = cudaFuncSetAttribute(tc::prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      tc::SMEM_BYTES)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(tc::prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      tc::SMEM_BYTES)) != cudaSuccess)
-            return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
+        const void* tc_kernels[4] = {reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, 128>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, 128>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, 64>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, 64>)};
+        for (const void* kern : tc_kernels)
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES)) !=
+                cudaSuccess)
+                return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
         if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
         d.attrs_set = true;
@@ -168,7 +171,7 @@ la_status check_dims(int dk, int dv, la_dtype dt) {
     return LA_OK;
 }
 
-bool use_tensor_cores(int d, la_dtype dt) { return dt == LA_BF16 && d == 128; }
+bool use_tensor_cores(int d, la_dtype dt) { return dt == LA_BF16 && (d == 128 || d == 64); }
 
 constexpr int kSimtDefaultChunk = 64;
 
@@ -186,15 +189,20 @@ la_status after_launch(const char* what) {
     return LA_OK;
 }
 
-// The tensor-core prefill, lean instance unless an option needs the general one.
+// The tensor-core prefill for p.dk (128 or 64), lean instance unless an
+// option needs the general one.
 la_status launch_tc(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
     const bool general =
         p.phi != LA_PHI_IDENTITY || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1);
-    if (general) tc::prefill_tc_kernel<true><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
-    else tc::prefill_tc_kernel<false><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    auto go = [&](auto kern) { kern<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p); };
+    if (p.dk == 64) general ? go(tc::prefill_tc_kernel<true, 64>) : go(tc::prefill_tc_kernel<false, 64>);
+    else general ? go(tc::prefill_tc_kernel<true, 128>) : go(tc::prefill_tc_kernel<false, 128>);
     return after_launch(what);
 }
+
+// (unit, value slice) work items per unit of the tensor-core prefill
+int tc_slices(int d) { return d / tc::DVS; }
 
 template <typename T, int D>
 void launch_simt_d(int cs, int grid, const void* q, const void* k, const void* v, void* o, const simt::Params& sp,
@@ -281,7 +289,7 @@ namespace {
 // SM remains.  LA_PREFILL_SEGMENTS=<n> overrides the count (1 = no split).
 constexpr int kMinSegChunks = 8;
 
-int plan_segments(long U, int N, int sms, int* seg_len) {
+int plan_segments(long U, int N, int d, int sms, int* seg_len) {
     const int nch = (N + tc::C - 1) / tc::C;
     *seg_len = nch * tc::C;
     if (N <= 0) return 1;
@@ -289,7 +297,7 @@ int plan_segments(long U, int N, int sms, int* seg_len) {
     if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
         P = atoi(e);
     } else {
-        const long items = U * tc::NVS;
+        const long items = U * (d / tc::DVS);
         P = items * 2 > sms ? 1 : (int)(sms / items);
         P = std::min(P, nch / kMinSegChunks);
     }
@@ -345,7 +353,7 @@ size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtyp
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return ph;
     int seg_len;
-    const size_t seg = segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), dk, dv);
+    const size_t seg = segment_workspace_bytes(U, plan_segments(U, N, dk, di->sms, &seg_len), dk, dv);
     return ph ? round256(seg) + ph : seg;
 }
 
@@ -383,9 +391,11 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         return launch_simt<__nv_bfloat16>(dk, chunk, (int)U, q, k, v, o, sp, st);
     }
 
+    const int nvs = tc_slices(dv);
     tc::Params p{};
     p.mode = 0;
-    p.n_items = (int)(U * tc::NVS);
+    p.dk = dk;
+    p.n_items = (int)(U * nvs);
     p.H = H;
     p.N = N;
     p.dv = dv;
@@ -397,11 +407,11 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     p.phi = phi;
     if (N == 0 && !s_out) return LA_OK;
     int seg_len;
-    int P = plan_segments(U, N, di->sms, &seg_len);
+    int P = plan_segments(U, N, dk, di->sms, &seg_len);
     p.seg_len = seg_len;
     const size_t ws_need = segment_workspace_bytes(U, P, dk, dv);
     if (P > 1 && (!workspace || ws_bytes < ws_need || !aligned16(workspace) ||
-                  (long)U * P * tc::NVS > (1L << 30))) {
+                  (long)U * P * nvs > (1L << 30))) {
         P = 1;  // no room for the segment states: one pass over whole sequences
         p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
     }
@@ -434,7 +444,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         float* starts = seg_sums + (size_t)U * (P - 1) * dk * dv;
         tc::Params p1 = p;
         p1.n_seg = P - 1;
-        p1.n_items = (int)(U * (P - 1) * tc::NVS);
+        p1.n_items = (int)(U * (P - 1) * nvs);
         p1.s0 = nullptr;
         p1.s_out = seg_sums;
         p1.s_out_per_seg = 1;
@@ -447,7 +457,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(seg_sums, s0, starts, U, P, dk * dv, 0, 0, dk);
         if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
         p.n_seg = P;
-        p.n_items = (int)(U * P * tc::NVS);
+        p.n_items = (int)(U * P * nvs);
         p.seg_init = starts;
     }
     const int grid = std::min(p.n_items, di->sms);
@@ -545,7 +555,8 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     p.mode = 1;
     p.n_seg = 1;
     p.phi = phi;
-    p.n_items = (int)((long)n_seq * H * tc::NVS);
+    p.dk = dk;
+    p.n_items = (int)((long)n_seq * H * tc_slices(dv));
     p.H = H;
     p.dv = dv;
     p.cu_seqlens = cu_seqlens;
@@ -724,9 +735,11 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
                                float* s_out, bool reverse, long U, int N, int d, DeviceInfo* di, cudaStream_t st,
                                void* ws, size_t ws_bytes) {
     if (N == 0 && !s_out) return LA_OK;
+    const int nvs = tc_slices(d);
     tc::Params p{};
     p.mode = 0;
-    p.n_items = (int)(U * tc::NVS);
+    p.dk = d;
+    p.n_items = (int)(U * nvs);
     p.N = N;
     p.dv = d;
     p.s0 = init;
@@ -738,9 +751,9 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     p.reverse = reverse ? 1 : 0;
     p.init_transposed = init_t ? 1 : 0;
     int seg_len;
-    int P = plan_segments(U, N, di->sms, &seg_len);
+    int P = plan_segments(U, N, d, di->sms, &seg_len);
     if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) ||
-                  U * P * tc::NVS > (1L << 30)))
+                  U * P * nvs > (1L << 30)))
         P = 1;
     p.seg_len = P > 1 ? seg_len : ((N + tc::C - 1) / tc::C) * tc::C;
     const void* any = N > 0 ? q : s_out;
@@ -757,7 +770,7 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
         tc::Params p1 = p;
         p1.n_seg = P - 1;
         p1.seg_base = reverse ? 1 : 0;  // the segments whose sums reach another segment's start
-        p1.n_items = (int)(U * (P - 1) * tc::NVS);
+        p1.n_items = (int)(U * (P - 1) * nvs);
         p1.s0 = nullptr;
         p1.init_transposed = 0;
         p1.s_out = sums;
@@ -772,7 +785,7 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
                                                                      init_t ? 1 : 0, d);
         if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
         p.n_seg = P;
-        p.n_items = (int)(U * P * tc::NVS);
+        p.n_items = (int)(U * P * nvs);
         p.seg_init = starts;
         p.init_transposed = 0;  // the segment starts are in the usual layout
     }
@@ -801,7 +814,7 @@ size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v,
     if (device_info(&di) != LA_OK) return 0;
     int seg_len;
     const long U = (long)B * H;
-    return segment_workspace_bytes(U, plan_segments(U, N, di->sms, &seg_len), d_k, d_v);
+    return segment_workspace_bytes(U, plan_segments(U, N, d_k, di->sms, &seg_len), d_k, d_v);
 }
 
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,

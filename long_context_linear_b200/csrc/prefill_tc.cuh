@@ -38,7 +38,7 @@ namespace lcl {
 namespace tc {
 
 constexpr int C = 128;         // chunk length (tokens)
-constexpr int DK = 128;        // key dim
+constexpr int DK = 128;        // largest key dim (the shared-memory layout is sized for it)
 constexpr int DVS = 64;        // value columns per CTA
 constexpr int Q_SLOTS = 2;
 constexpr int K_SLOTS = 2;
@@ -79,7 +79,7 @@ static_assert((BAR_COUNT + 2) * 8 <= BAR_BYTES, "barrier area too small");
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB per-block shared memory limit");
 constexpr int NUM_THREADS = 512;
-constexpr int NVS = 2;          // value slices per head (d_v = 128 on this path)
+// value slices per head: d_v / DVS (2 at d = 128, 1 at d = 64; d_k = d_v)
 constexpr int WARP_MMA_A = 1;
 constexpr int WARP_MMA_B = 14;
 constexpr int WARP_LOAD_V = 15;
@@ -96,7 +96,7 @@ struct Params {
     int n_items;           // work items
     int H;                 // heads (packed layout)
     int N;                 // tokens per unit (dense)
-    int dv;                // full value dim (= NVS * DVS)
+    int dv;                // full value dim (= slices * DVS), equal to the key dim
     const int* cu_seqlens; // packed: [n_seq + 1]
     const int* order;      // packed: sequence indices, longest first
     const float* s0;       // dense: [U][DK][dv] or null
@@ -118,6 +118,7 @@ struct Params {
     int reverse;
     int init_transposed;   // the initial state is given as its transpose [dv][DK]
     int seg_base;          // dense: the items' segments are seg_base .. seg_base + n_seg - 1
+    int dk;                // key dim = value dim: 128 or 64 (selects the kernel instance)
 };
 
 struct Item {
@@ -139,22 +140,23 @@ __device__ __forceinline__ int item_index(int round, int cta, int grid) {
 // First token (relative to the item's start) of the c-th chunk in visiting order.
 __device__ __forceinline__ int chunk_row(bool rev, int c, int nc) { return (rev ? nc - 1 - c : c) * C; }
 
-// kGeneral = false: dense items are whole sequences (n_seg = 1).
-template <bool kGeneral>
+// kGeneral = false: dense items are whole sequences (n_seg = 1).  KD: key dim.
+template <bool kGeneral, int KD>
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
+    constexpr int NV = KD / DVS;  // value slices per unit
     Item it;
-    it.vs = idx & (NVS - 1);
+    it.vs = idx % NV;
     if (!kGeneral && p.mode == 0) {
-        const int u = idx / NVS;
+        const int u = idx / NV;
         it.t0 = 0;
         it.len = p.N;
         it.c1 = 0;
         it.c2 = u;
         it.state = u;
-        it.init = p.s0 ? p.s0 + (long)u * DK * p.dv : nullptr;
+        it.init = p.s0 ? p.s0 + (long)u * KD * p.dv : nullptr;
         it.write_state = true;
     } else if (p.mode == 0) {
-        const int us = idx / NVS;  // unit * n_seg + segment
+        const int us = idx / NV;  // unit * n_seg + segment
         const int u = us / p.n_seg, sg = us - u * p.n_seg;
         // the segment visited first starts from s0; the one visited last ends the sequence
         const int first = p.reverse ? p.n_seg - 1 : 0, last = p.reverse ? 0 : p.n_seg - 1;
@@ -163,11 +165,11 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
         it.c1 = 0;
         it.c2 = u;
         it.state = p.s_out_per_seg ? us : u;
-        it.init = p.seg_init ? p.seg_init + (long)us * DK * p.dv
-                             : ((sg == first && p.s0) ? p.s0 + (long)u * DK * p.dv : nullptr);
+        it.init = p.seg_init ? p.seg_init + (long)us * KD * p.dv
+                             : ((sg == first && p.s0) ? p.s0 + (long)u * KD * p.dv : nullptr);
         it.write_state = p.s_out_per_seg || sg == last;
     } else {
-        const int hs = idx / NVS;   // sequence rank * H + head
+        const int hs = idx / NV;    // sequence rank * H + head
         const int r = hs / p.H;
         const int h = hs - r * p.H;
         const int seq = p.order ? p.order[r] : r;
@@ -177,7 +179,7 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
         it.c2 = 0;
         it.state = (long)seq * p.H + h;
         const int ii = p.init_idx ? p.init_idx[seq] : -1;
-        it.init = (p.pool && ii >= 0) ? p.pool + ((long)ii * p.H + h) * DK * p.dv : nullptr;
+        it.init = (p.pool && ii >= 0) ? p.pool + ((long)ii * p.H + h) * KD * p.dv : nullptr;
         it.write_state = true;
     }
     return it;
@@ -256,8 +258,9 @@ __device__ __forceinline__ constexpr uint64_t mnmaj_step(int kk) { return static
 // kGeneral = false is the lean instance for the common case (feature map
 // identity, chunks in order, outputs computed, initial state as given, whole
 // sequences): the options below are then compile-time constants and their
-// code is left out.
-template <bool kGeneral>
+// code is left out.  KD = d_k = d_v: 128 (two 64-column panels per Q and K
+// tile, two value slices per head) or 64 (one panel, one slice).
+template <bool kGeneral, int KD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -293,6 +296,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int phi = kGeneral ? p.phi : static_cast<int>(PHI_IDENTITY);
     const bool rev = kGeneral && p.reverse;
     const bool init_t = kGeneral && p.init_transposed;
+    constexpr int NP = KD / 64;  // 64-column panels per Q / K tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < Q_SLOTS; ++i) {
@@ -345,7 +349,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item<kGeneral>(p, idx);
+                const Item it = decode_item<kGeneral, KD>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 // chunk c is brought into L2 PREFETCH chunks before its load
                 for (int c = -PREFETCH; c < nc; ++c) {
@@ -353,12 +357,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     if (cp < nc) {
                         const int t = it.t0 + chunk_row(rev, cp, nc);
                         const int y = p.mode == 0 ? t : it.c1, z = p.mode == 0 ? it.c2 : t;
-                        if (!state_only) {
-                            tma_prefetch_3d(&map_q, 0, y, z);
-                            tma_prefetch_3d(&map_q, 64, y, z);
+#pragma unroll
+                        for (int pn = 0; pn < NP; ++pn) {
+                            if (!state_only) tma_prefetch_3d(&map_q, 64 * pn, y, z);
+                            tma_prefetch_3d(&map_k, 64 * pn, y, z);
                         }
-                        tma_prefetch_3d(&map_k, 0, y, z);
-                        tma_prefetch_3d(&map_k, 64, y, z);
                         tma_prefetch_3d(&map_v, DVS * it.vs, y, z);
                     }
                     if (c < 0) continue;
@@ -368,16 +371,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     if (!state_only) {
                         if (kq > 0 && !mbar_wait(&q_empty[qs], (kq - 1) & 1, abort, p.status)) { stop = true; break; }
                         uint8_t* qb = sm + OFF_Q + qs * TILE_Q;
-                        mbar_arrive_expect_tx(&q_full[qs], TILE_Q);
-                        tma_load_3d(qb, &map_q, &q_full[qs], 0, y, z);
-                        tma_load_3d(qb + PANEL, &map_q, &q_full[qs], 64, y, z);
+                        mbar_arrive_expect_tx(&q_full[qs], NP * PANEL);
+#pragma unroll
+                        for (int pn = 0; pn < NP; ++pn) tma_load_3d(qb + pn * PANEL, &map_q, &q_full[qs], 64 * pn, y, z);
                     }
                     const int ks = g % K_SLOTS, kk_ = g / K_SLOTS;
                     if (kk_ > 0 && !mbar_wait(&k_empty[ks], (kk_ - 1) & 1, abort, p.status)) { stop = true; break; }
                     uint8_t* kb = sm + OFF_K + ks * TILE_K;
-                    mbar_arrive_expect_tx(&k_full[ks], 2 * PANEL);
-                    tma_load_3d(kb, &map_k, &k_full[ks], 0, y, z);
-                    tma_load_3d(kb + KPANEL, &map_k, &k_full[ks], 64, y, z);
+                    mbar_arrive_expect_tx(&k_full[ks], NP * PANEL);
+#pragma unroll
+                    for (int pn = 0; pn < NP; ++pn) tma_load_3d(kb + pn * KPANEL, &map_k, &k_full[ks], 64 * pn, y, z);
                     ++g;
                 }
             }
@@ -395,7 +398,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item<kGeneral>(p, idx);
+                const Item it = decode_item<kGeneral, KD>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
                     const int t = it.t0 + chunk_row(rev, c, nc);
@@ -423,7 +426,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0;; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                total += (decode_item<kGeneral>(p, idx).len + C - 1) / C;
+                total += (decode_item<kGeneral, KD>(p, idx).len + C - 1) / C;
             }
             int k = 0;  // next chunk whose [P|O] is to be issued
             int g = 0;  // chunk whose P V is issued next
@@ -431,7 +434,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item<kGeneral>(p, idx).len;
+                const int len = decode_item<kGeneral, KD>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     // [P | O] = Q [K ; S^T]^T for chunks up to g + 1  (A: Q, B: K rows then S^T rows)
                     for (; k <= g + 1 && k < total; ++k) {
@@ -442,7 +445,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         const uint64_t da = kmaj_desc(sq + qs * TILE_Q, 0, PANEL);
                         const uint64_t db = kmaj_desc(sk + ks * TILE_K, 0, KPANEL);
 #pragma unroll
-                        for (int kk = 0; kk < DK / 16; ++kk)
+                        for (int kk = 0; kk < KD / 16; ++kk)
                             mma_ss(tpo, da + kmaj_step(kk, PANEL), db + kmaj_step(kk, KPANEL), id_f, kk > 0);
                         mma_commit(&p_full[b]);
                         mma_commit(&q_empty[qs]);
@@ -488,7 +491,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item<kGeneral>(p, idx).len;
+                const int len = decode_item<kGeneral, KD>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     const int ks = g % K_SLOTS, vc = g % V_SLOTS, b = g & 1;
                     const int rows = len - c0;
@@ -501,7 +504,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     if (g >= 2 && !mbar_wait(&ds_empty[b], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }
                     tc_fence_after();
                     const uint32_t tds = tbase + TM_DS + TM_PO_STRIDE * b;
-                    const uint64_t dk = mnmaj_desc(sk + ks * TILE_K, 0, KPANEL), dv = mnmaj_desc(sv + vc * PANEL, 0, PANEL);
+                    // A = K^T, 128 rows of key dims: at d = 64 the second 64-row half reads
+                    // the same panel again (leading offset 0), so dS rows 64..127 repeat
+                    // rows 0..63 and are ignored
+                    const uint64_t dk = mnmaj_desc(sk + ks * TILE_K, 0, KD == 128 ? KPANEL : 0),
+                                   dv = mnmaj_desc(sv + vc * PANEL, 0, PANEL);
                     if (ksteps == C / 16) {
 #pragma unroll
                         for (int kk = 0; kk < C / 16; ++kk) mma_ss(tds, dk + mnmaj_step(kk), dv + mnmaj_step(kk), id_ds, kk > 0);
@@ -533,7 +540,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const int len = decode_item<kGeneral>(p, idx).len;
+                const int len = decode_item<kGeneral, KD>(p, idx).len;
                 for (int c0 = 0; c0 < len; c0 += C, ++g) {
                     const int b = g & 1;
                     if (!warp_wait(&p_full[b], (g >> 1) & 1, abort, p.status)) { stop = true; break; }
@@ -571,6 +578,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // ------------------------------------------------------ state warps
         const int q4 = warp & 3;
         const int i = q4 * 32 + lane;  // key-dim row of S owned by this thread
+        const bool own = KD == 128 || q4 < KD / 32;  // warp-uniform; at d = 64 warps 8, 9 only follow along
         const uint32_t ta0 = tbase + (static_cast<uint32_t>(q4 * 32) << 16) + TM_DS;
         // S^T row j (value column j) sits at row C + j of each K panel; this
         // thread writes the bf16 of S[i][j] at dk column i of every row.  A
@@ -582,14 +590,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         for (int r = 0; !stop; ++r) {
             const int idx = item_index(r, cta, G);
             if (idx >= p.n_items) break;
-            const Item it = decode_item<kGeneral>(p, idx);
+            const Item it = decode_item<kGeneral, KD>(p, idx);
             float S[DVS];
-            if (it.init && init_t) {
+            if (it.init && init_t && own) {
                 // column i of rows DVS vs .. DVS vs + DVS - 1 of the transposed block
-                const float* src = it.init + (long)DVS * it.vs * DK + i;
+                const float* src = it.init + (long)DVS * it.vs * KD + i;
 #pragma unroll
-                for (int j = 0; j < DVS; ++j) S[j] = src[j * DK];
-            } else if (it.init) {
+                for (int j = 0; j < DVS; ++j) S[j] = src[j * KD];
+            } else if (it.init && own) {
                 const float4* src = reinterpret_cast<const float4*>(it.init + (long)i * p.dv + DVS * it.vs);
 #pragma unroll
                 for (int j = 0; j < DVS / 4; ++j) {
@@ -605,13 +613,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const int ks = g % K_SLOTS;
                 if (!state_only) {
                     if (g >= K_SLOTS && !warp_wait(&k_empty[ks], ((g / K_SLOTS) - 1) & 1, abort, p.status)) { stop = true; break; }
-                    uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
-                    __nv_bfloat16* rowp[8];
+                    if (own) {
+                        uint8_t* base = sm + OFF_K + ks * TILE_K + col_off;
+                        __nv_bfloat16* rowp[8];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m)
-                        rowp[m] = reinterpret_cast<__nv_bfloat16*>(base + ((colchunk ^ static_cast<uint32_t>(m)) << 4));
+                        for (int m = 0; m < 8; ++m)
+                            rowp[m] = reinterpret_cast<__nv_bfloat16*>(base + ((colchunk ^ static_cast<uint32_t>(m)) << 4));
 #pragma unroll
-                    for (int j = 0; j < DVS; ++j) rowp[j & 7][j * 64] = __float2bfloat16_rn(S[j]);
+                        for (int j = 0; j < DVS; ++j) rowp[j & 7][j * 64] = __float2bfloat16_rn(S[j]);
+                    }
                     fence_proxy_async_smem();
                     // the [P|O] product of this chunk also needs Q_c, K_c and the O
                     // buffer it writes (last used by chunk c - 2) drained
@@ -624,11 +634,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     // phi(K_c), then phi(Q_c), in place, before the tensor cores read
                     // them (the S^T rows behind K are left alone); K first, so that
                     // K^T V can start while Q is mapped
-                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, 2 * PANEL / 16, i, phi);
+                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, NP * PANEL / 16, i, phi);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&kphi_full[ks]);
                     if (!state_only)
-                        phi_region(smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q), PANEL, PANEL / 16, 2 * PANEL / 16, i,
+                        phi_region(smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q), PANEL, PANEL / 16, NP * PANEL / 16, i,
                                    phi);
                 }
                 if (!state_only) {
@@ -654,8 +664,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (lane == 0) mbar_arrive(&ds_empty[b]);
             }
             if (stop) break;
-            if (p.s_out && it.write_state) {
-                float4* dst = reinterpret_cast<float4*>(p.s_out + (it.state * DK + i) * p.dv + DVS * it.vs);
+            if (p.s_out && it.write_state && own) {
+                float4* dst = reinterpret_cast<float4*>(p.s_out + (it.state * KD + i) * p.dv + DVS * it.vs);
 #pragma unroll
                 for (int j = 0; j < DVS / 4; ++j)
                     dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
@@ -672,7 +682,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int r = 0; !stop; ++r) {
                 const int idx = item_index(r, cta, G);
                 if (idx >= p.n_items) break;
-                const Item it = decode_item<kGeneral>(p, idx);
+                const Item it = decode_item<kGeneral, KD>(p, idx);
                 const int nc = (it.len + C - 1) / C;
                 for (int c = 0; c < nc; ++c, ++g) {
                     const int c0 = chunk_row(rev, c, nc);

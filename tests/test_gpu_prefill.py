@@ -169,3 +169,28 @@ def test_tc_many_units_per_cta(la, oracle_mod):
     ro, rs = oracle_mod.recurrent(qf[idx], kf[idx], vf[idx], s0f[idx])
     assert_out(of[idx], ro, torch.bfloat16, 1)
     assert_state(sf[idx], rs, 1)
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 1, 1), (2, 3, 300), (1, 2, 1000), (3, 1, 4096 + 5)])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_tc_d64_matches_oracle(la, oracle_mod, B, H, N, with_s0):
+    """d = 64 on the tensor cores: one 64-column panel, one value slice per
+    head, the K^T V product's second half a copy of the first."""
+    q, k, v = synth.dense(B, H, N, 64, "bf16", seed=B * 7 + H + N)
+    s0 = _state(B, H, 64, seed=N) if with_s0 else None
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.bfloat16, 2)
+    assert_state(s, rs, 2)
+
+
+def test_tc_d64_integer_inputs_bit_exact(la, oracle_mod):
+    B, H, N, d = 2, 2, 1000, 64
+    q = synth.integer_valued((B, H, N, d), seed=51, dtype=torch.bfloat16)
+    k = synth.integer_valued((B, H, N, d), seed=52, dtype=torch.bfloat16)
+    v = synth.integer_valued((B, H, N, d), seed=53, dtype=torch.bfloat16)
+    s0 = synth.integer_valued((B, H, d, d), seed=54, lo=-20, hi=20, dtype=torch.float32)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert torch.equal(o, torch.from_numpy(ro).to(torch.bfloat16))
+    np.testing.assert_array_equal(to64(s), rs)

@@ -107,3 +107,15 @@ def test_workspace_size_follows_the_plan(la):
     # one head over 64K tokens: (2P - 1) fp32 states of 128 x 128
     n = la.prefill_workspace_size(1, 1, 65536, 128, torch.bfloat16)
     assert n > 0 and n % (128 * 128 * 4) == 0 and (n // (128 * 128 * 4)) % 2 == 1
+
+
+@pytest.mark.parametrize("segments", ["1", "3"])
+def test_segments_d64(la, oracle_mod, monkeypatch, segments):
+    """The segment split at d = 64 (one value slice per unit)."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v = synth.dense(1, 2, 5000, 64, "bf16", seed=91)
+    s0 = _state(1, 2, 64, seed=92)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.bfloat16, 2)
+    assert_state(s, rs, 2)
