@@ -1,8 +1,8 @@
 """Gradients of the prefill (la_prefill_backward) against the fp64 oracle's
 chain rule through the recurrence (itself pinned to finite differences and to
-autograd of the quadratic form in tests/test_oracle.py).  bf16 with d = 128
-runs three tensor-core passes (two of them in reverse token order); fp32, d =
-64 and LA_BACKWARD_SIMT=1 run the FFMA kernel."""
+autograd of the quadratic form in tests/test_oracle.py).  bf16 (d = 128 or
+64) runs three tensor-core passes (two of them in reverse token order); fp32
+and LA_BACKWARD_SIMT=1 run the same passes on the FFMA kernel."""
 import numpy as np
 import pytest
 import torch

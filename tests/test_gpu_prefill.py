@@ -1,5 +1,5 @@
-"""Dense prefill on the GPU against the fp64 oracle (tensor-core bf16 path and
-the FFMA fp32 / d=64 path), through the C ABI via the Python binding."""
+"""Dense prefill on the GPU against the fp64 oracle (tensor-core bf16 path at
+d = 128 and 64, FFMA fp32 path), through the C ABI via the Python binding."""
 import numpy as np
 import pytest
 import torch
