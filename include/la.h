@@ -30,9 +30,9 @@
  *  - Alignment: every tensor pointer must be 16-byte aligned.
  *  - Aliasing: no input may alias an output, except the in-place state of
  *    la_decode_step.
- *  - Dimensions: d_k = d_v = d with d in {64, 128}.  bf16 inputs with d = 128
- *    run on the tcgen05 tensor-core path; fp32 inputs and d = 64 run on a
- *    CUDA-core FFMA path.  Anything else returns LA_ERR_UNSUPPORTED.
+ *  - Dimensions: d_k = d_v = d with d in {64, 128}.  bf16 inputs run on the
+ *    tcgen05 tensor-core path; fp32 inputs run on a CUDA-core FFMA path.
+ *    Anything else returns LA_ERR_UNSUPPORTED.
  *  - Output dtype equals the input dtype; states are always fp32.
  *  - Device-side waits are bounded; a wait that runs out records
  *    LA_ERR_TIMEOUT in a device status word read by la_device_status().
@@ -251,10 +251,10 @@ LA_API la_status la_prefill_host(const void* q, const void* k, const void* v, vo
  * S carried forward for dq and G carried backward for dk, dv).
  *   q, k, dq, dk : [B, H, N, d_k];  v, dout, dv : [B, H, N, d_v]   dtype `dt`
  *   s0, ds_n     : fp32 [B, H, d_k, d_v] or NULL (zero);  ds0: fp32 or NULL.
- * bf16 with d = 128: three tensor-core passes of the prefill kernel
+ * bf16 (d = 128 or 64): three tensor-core passes of the prefill kernel
  * (dq = prefill(dout, v, k) from s0^T; dk = prefill(v, dout, q) from ds_n^T
  * and dv = prefill(k, q, dout) from ds_n, both with time reversed), with the
- * prefill's precision.  fp32 or d = 64: the same three passes on the FFMA
+ * prefill's precision.  fp32: the same three passes on the FFMA
  * prefill kernel, fp32 arithmetic.
  * d_k = d_v in {64, 128}.  All pointers 16-byte aligned; the caller owns every
  * buffer; no host synchronisation.  Errors: LA_ERR_INVALID_ARG (null, negative,
