@@ -445,11 +445,12 @@ def run_varlen(args, dist: Dist, pk):
                 frac=gbs / pk["hbm"], tflops_rec=flops_rec(T * H, d) / (ms_step / 1e3) / 1e12, steps=n)
 
 
-def run_prefill8k(args, dist: Dist, pk, phi: str = "identity"):
+def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0):
     import long_context_linear_b200 as la
     import synth
     c = PREFILL8K
-    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    B, H, N = c["B"], c["H"], c["N"]
+    d = d or c["d"]
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = synth.dense(B, H, N, d, "bf16", seed=61 + dist.rank, device=dev)
     o = torch.empty_like(v)
@@ -467,11 +468,11 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity"):
     gbs = byts / (ms_step / 1e3) / 1e9
     del q, k, v, o, s, ws
     torch.cuda.empty_cache()
-    return dict(workload=f"prefill B=4 H=32 N=8192 d=128 bf16, feature map {phi}",
+    return dict(workload=f"prefill B=4 H=32 N=8192 d={d} bf16, feature map {phi}",
                 tokens_per_s=B * N * dist.world / (ms_step / 1e3),
                 ms_per_step=ms_step, hbm_gbs=gbs, frac=gbs / pk["hbm"],
                 tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
-                l2="inputs (1 GiB) larger than L2")
+                l2="inputs (%.0f MiB) larger than L2" % (3 * B * H * N * d * 2 / 2**20))
 
 
 def run_backward(args, dist: Dist, pk):
@@ -662,6 +663,7 @@ def main():
         extras["varlen"] = run_varlen(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
+        extras["prefill_8k_d64"] = run_prefill8k(args, dist, pk, d=64)
         extras["few_heads"] = run_few_heads(args, dist, pk)
         extras["backward_8k"] = run_backward(args, dist, pk)
     cpu = None
