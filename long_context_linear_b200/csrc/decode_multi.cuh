@@ -31,6 +31,19 @@ constexpr int MAX_M = 16;
 
 constexpr int G = 4;  // draft tokens per reduction round of verify
 
+// 16 bytes of T -> fp32 (4 fp32 or 8 bf16 values)
+__device__ __forceinline__ void unpack16(const uint4 r, float (&f)[4]) {
+    f[0] = __uint_as_float(r.x); f[1] = __uint_as_float(r.y); f[2] = __uint_as_float(r.z); f[3] = __uint_as_float(r.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 r, float (&f)[8]) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
 // Two CTAs per SM: the bound lets the compiler use up to 128 registers, and
 // with them verify keeps more loads in flight (measured: 0.213 ms against
 // 0.257 ms at 101 registers for B=256, H=64, m=4).
@@ -41,9 +54,9 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     constexpr int TPR = D / 4;
     constexpr int RS = NUM_THREADS / TPR;
     constexpr int RPT = D / RS;
-    __shared__ float qs[MAX_M][D], ks[MAX_M][D], vs[MAX_M][D];
+    __shared__ __align__(16) float qs[MAX_M][D], ks[MAX_M][D], vs[MAX_M][D];
     __shared__ float A[MAX_M][MAX_M];  // A[t][s] = q_t . k_s, s <= t
-    __shared__ float red[G][RS][D];
+    __shared__ __align__(16) float red[G][RS][D];
 
     const long u = blockIdx.x;
     const int tid = threadIdx.x;
@@ -53,26 +66,41 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 #pragma unroll
     for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
     const long base = u * (long)m * D;
-    for (int e = tid; e < m * D; e += NUM_THREADS) {
-        qs[e / D][e % D] = apply_phi(dec::ld_f(q + base + e), phi);
-        ks[e / D][e % D] = apply_phi(dec::ld_f(k + base + e), phi);
-        vs[e / D][e % D] = dec::ld_f(v + base + e);
+    // the drafts' q, k, v: 16-byte loads (rows are 16-byte aligned: D * sizeof(T) is)
+    constexpr int VEC = 16 / (int)sizeof(T);
+    for (int e = tid * VEC; e < m * D; e += NUM_THREADS * VEC) {
+        const int t = e / D, i = e % D;
+        float qv[VEC], kv[VEC], vv[VEC];
+        unpack16(*reinterpret_cast<const uint4*>(q + base + e), qv);
+        unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
+        unpack16(*reinterpret_cast<const uint4*>(v + base + e), vv);
+#pragma unroll
+        for (int j = 0; j < VEC; j += 4) {
+            *reinterpret_cast<float4*>(&qs[t][i + j]) = make_float4(apply_phi(qv[j], phi), apply_phi(qv[j + 1], phi),
+                                                                    apply_phi(qv[j + 2], phi), apply_phi(qv[j + 3], phi));
+            *reinterpret_cast<float4*>(&ks[t][i + j]) = make_float4(apply_phi(kv[j], phi), apply_phi(kv[j + 1], phi),
+                                                                    apply_phi(kv[j + 2], phi), apply_phi(kv[j + 3], phi));
+            *reinterpret_cast<float4*>(&vs[t][i + j]) = make_float4(vv[j], vv[j + 1], vv[j + 2], vv[j + 3]);
+        }
     }
     __syncthreads();
-    // intra-draft scores: one warp per pair (t, s), s <= t, lanes split the dim
+    // intra-draft scores: one warp per pair (t, s), s <= t, lanes split the dim;
+    // pairs in row order, warp w taking every 8th from the w-th, (t, s) stepped
+    // along without recomputing it from the pair index
     {
+        constexpr int NW = NUM_THREADS / 32;
         const int warp = tid >> 5, lane = tid & 31;
-        const int np = m * (m + 1) / 2;
-        for (int pi = warp; pi < np; pi += NUM_THREADS / 32) {
-            int t = 0;
-            while ((t + 1) * (t + 2) / 2 <= pi) ++t;
-            const int s = pi - t * (t + 1) / 2;
+        int t = 0, s = warp;
+        while (s > t) { s -= t + 1; ++t; }
+        for (; t < m;) {
             float a = 0.f;
 #pragma unroll
             for (int i = lane; i < D; i += 32) a = fmaf(qs[t][i], ks[s][i], a);
 #pragma unroll
             for (int off = 16; off; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
             if (lane == 0) A[t][s] = a;
+            s += NW;
+            while (s > t) { s -= t + 1; ++t; }
         }
     }
     // q_t S_0 for G draft tokens at a time, reduced over row slots, plus the
@@ -117,7 +145,7 @@ commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restric
     constexpr int TPR = D / 4;
     constexpr int RS = NUM_THREADS / TPR;
     constexpr int RPT = D / RS;
-    __shared__ float ks[MAX_M][D], vs[MAX_M][D];
+    __shared__ __align__(16) float ks[MAX_M][D], vs[MAX_M][D];
 
     const long u = blockIdx.x;
     const int tid = threadIdx.x;
