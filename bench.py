@@ -50,8 +50,8 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "5930f87d59086621"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.75e6 + 116.02e6) / (16 * 32768)
+TRAFFIC_HASH = "3c28761b61fecc54"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.98e6 + 113.45e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
