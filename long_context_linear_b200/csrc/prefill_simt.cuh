@@ -40,12 +40,6 @@ struct Params {
     int init_transposed;    // the initial state is given as its transpose [d][d]
 };
 
-__device__ __forceinline__ float to_f(float x) { return x; }
-__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename T> __device__ __forceinline__ T from_f(float x);
-template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
-
 // Shared-memory layout (floats), rows padded by 4 so that 16-byte vectors
 // stay aligned and successive rows start in different banks:
 //   Qt, Kt [D][CS+4]   Q and K transposed (token index contiguous)
