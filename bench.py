@@ -103,6 +103,17 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def bad_clocks(c) -> bool:
+    """hw_slowdown / hw_thermal_slowdown / sw_thermal_slowdown active, or the
+    median SM clock under load below 60 % of its maximum with no reason
+    active; sw_power_cap alone is expected under load and kept."""
+    reasons = set(c.get("reasons") or [])
+    if reasons & {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}:
+        return True
+    sm, mx = c.get("sm_mhz"), c.get("sm_max_mhz")
+    return bool(sm and mx and not reasons and sm < 0.6 * mx)
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples for one GPU while a region runs."""
 
@@ -651,6 +662,15 @@ def main():
     pk = peaks()
     sampler = ClockSampler(dist.local)
     head, _ = run_headline(args, dist, pk, sampler)
+    # a run that saw hardware or thermal slowdown, or SM clocks held far below
+    # their maximum with no reason given (a leftover clock lock), is measured
+    # once more; every rank takes the same decision
+    bad = bad_clocks(head["clocks"])
+    if dist.max(1.0 if bad else 0.0) > 0:
+        print(f"note: clocks {head['clocks']} -> measuring the headline once more", file=sys.stderr)
+        first = head["clocks"]
+        head, _ = run_headline(args, dist, pk, sampler)
+        head["clocks"]["remeasured_after"] = dict(reasons=first.get("reasons"), sm_mhz=first.get("sm_mhz"))
     extras = {}
     if not args.no_extras:
         extras["decode"] = run_decode(args, dist, pk)
