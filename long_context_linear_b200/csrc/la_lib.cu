@@ -279,7 +279,7 @@ const char* la_status_string(la_status s) {
 
 const char* la_last_error(void) { return g_last_error; }
 
-int la_version(void) { return 100; }
+int la_version(void) { return 200; }  // 0.2.0
 
 namespace {
 
