@@ -123,11 +123,12 @@ struct VecFp8 {
 template <> struct Vec<__nv_fp8_e4m3> : VecFp8<__NV_E4M3> {};
 template <> struct Vec<__nv_fp8_e5m2> : VecFp8<__NV_E5M2> {};
 
-// Threads per CTA: an 8-bit state is 16 KB per unit at d = 128, so its CTAs
-// are half as wide and twice as many units are in flight per SM (measured on
-// B=256, H=64: 5.34 TB/s at 128 threads, 3.34 at 256, 4.46 at 64).
+// Threads per CTA: 16- and 8-bit states are 32 / 16 KB per unit at d = 128,
+// so their CTAs are half as wide and twice as many units are in flight per SM
+// (measured on B=256, H=64: fp8 5.34 TB/s at 128 threads, 3.34 at 256, 4.46
+// at 64; bf16 6.72 TB/s at 128 threads, 6.56 at 256).
 template <typename SS>
-__host__ __device__ constexpr int decode_threads() { return Vec<SS>::E == 16 ? NUM_THREADS / 2 : NUM_THREADS; }
+__host__ __device__ constexpr int decode_threads() { return Vec<SS>::E >= 8 ? NUM_THREADS / 2 : NUM_THREADS; }
 
 template <typename T, typename SS, int D>
 __global__ void __launch_bounds__(decode_threads<SS>())
