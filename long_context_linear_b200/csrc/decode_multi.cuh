@@ -136,10 +136,9 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
 }
 
-// MINB = 3 (a few registers spilled) pays off from m > 8 drafts on, where
-// each CTA spends longer on its rank-1 updates; below that MINB = 2.
-template <typename T, int D, int MINB>
-__global__ void __launch_bounds__(NUM_THREADS, MINB)
+// Two CTAs per SM (up to 128 registers, no spills).
+template <typename T, int D>
+__global__ void __launch_bounds__(NUM_THREADS, 2)
 commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restrict__ S,
               const int* __restrict__ accepted, int H, int m, int phi) {
     constexpr int TPR = D / 4;
@@ -150,16 +149,28 @@ commit_kernel(const T* __restrict__ k, const T* __restrict__ v, float* __restric
     const long u = blockIdx.x;
     const int tid = threadIdx.x;
     const int c4 = tid % TPR, slot = tid / TPR;
-    const int a = min(max(accepted[u / H], 0), m);
-    if (a == 0) return;
+    // the state loads go out before the accepted count is known, so that the
+    // two memory latencies overlap (a unit that accepts nothing reads its
+    // state in vain)
     float4* Su = reinterpret_cast<float4*>(S + u * D * D);
     float4 x[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
+    const int a = min(max(accepted[u / H], 0), m);
+    if (a == 0) return;
     const long base = u * (long)m * D;
-    for (int e = tid; e < a * D; e += NUM_THREADS) {
-        ks[e / D][e % D] = apply_phi(dec::ld_f(k + base + e), phi);
-        vs[e / D][e % D] = dec::ld_f(v + base + e);
+    constexpr int VEC = 16 / (int)sizeof(T);
+    for (int e = tid * VEC; e < a * D; e += NUM_THREADS * VEC) {
+        const int t = e / D, i = e % D;
+        float kv[VEC], vv[VEC];
+        unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
+        unpack16(*reinterpret_cast<const uint4*>(v + base + e), vv);
+#pragma unroll
+        for (int j = 0; j < VEC; j += 4) {
+            *reinterpret_cast<float4*>(&ks[t][i + j]) = make_float4(apply_phi(kv[j], phi), apply_phi(kv[j + 1], phi),
+                                                                    apply_phi(kv[j + 2], phi), apply_phi(kv[j + 3], phi));
+            *reinterpret_cast<float4*>(&vs[t][i + j]) = make_float4(vv[j], vv[j + 1], vv[j + 2], vv[j + 3]);
+        }
     }
     __syncthreads();
     for (int t = 0; t < a; ++t) {

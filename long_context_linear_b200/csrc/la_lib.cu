@@ -248,8 +248,7 @@ namespace {
 template <typename T, int D>
 void launch_commit_d(int m, int grid, const T* k, const T* v, float* S, const int32_t* accepted, int H, int phi,
                      cudaStream_t st) {
-    if (m > 8) dmulti::commit_kernel<T, D, 3><<<grid, dmulti::NUM_THREADS, 0, st>>>(k, v, S, accepted, H, m, phi);
-    else dmulti::commit_kernel<T, D, 2><<<grid, dmulti::NUM_THREADS, 0, st>>>(k, v, S, accepted, H, m, phi);
+    dmulti::commit_kernel<T, D><<<grid, dmulti::NUM_THREADS, 0, st>>>(k, v, S, accepted, H, m, phi);
 }
 
 template <typename T>
