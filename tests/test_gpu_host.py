@@ -28,6 +28,7 @@ def _pinned(t):
     (1, 16, 4096, 128, "bf16", 4, True),
     (1, 4, 777, 128, "bf16", 64, False),     # one group larger than the batch
     (2, 2, 200, 64, "fp32", 1, True),        # FFMA path, one unit per group
+    (2, 3, 500, 64, "bf16", 4, True),        # tensor cores at d = 64
 ])
 def test_host_prefill_equals_device_prefill(la, monkeypatch, B, H, N, d, dtype, group, with_s0):
     monkeypatch.setenv("LA_PREFILL_SEGMENTS", "1")  # the reference in one pass, as every host group runs
