@@ -486,6 +486,46 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0):
                 l2="inputs (%.0f MiB) larger than L2" % (3 * B * H * N * d * 2 / 2**20))
 
 
+def run_varlen_few(args, dist: Dist, pk):
+    """A packed batch of two 64K-token sequences with H=8 (32 items on 148
+    SMs), with and without the segment split."""
+    import long_context_linear_b200 as la
+    import synth
+    lens, H, d = [65536, 65536], 8, 128
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cu = synth.cu_seqlens(lens).to(dev)
+    T = sum(lens)
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=87 + dist.rank, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(len(lens), H, d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(la.prefill_varlen_workspace_size(len(lens), T, H, d, torch.bfloat16), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = max(10, min(args.steps, 50))
+    byts = 4.0 * T * H * d * 2 + len(lens) * H * d * d * 4
+    res = dict(workload="varlen 2 sequences x 65536 tokens, H=8, d=128, bf16", workspace_bytes=ws.numel(), steps=n)
+    prev = os.environ.get("LA_PREFILL_SEGMENTS")
+    try:
+        for key, env in (("split", None), ("unsplit", "1")):
+            if env is None:
+                os.environ.pop("LA_PREFILL_SEGMENTS", None)
+            else:
+                os.environ["LA_PREFILL_SEGMENTS"] = env
+            total_ms, _ = timed_launches(lambda: la.prefill_varlen(q, k, v, cu, out=o, s_out=s, workspace=ws), n,
+                                         max(3, args.warmup), dist, stream)
+            ms_step = dist.max(total_ms) / n
+            res[key] = dict(ms_per_step=ms_step, hbm_gbs=byts / (ms_step / 1e3) / 1e9,
+                            frac=byts / (ms_step / 1e3) / 1e9 / pk["hbm"])
+    finally:
+        if prev is None:
+            os.environ.pop("LA_PREFILL_SEGMENTS", None)
+        else:
+            os.environ["LA_PREFILL_SEGMENTS"] = prev
+    del q, k, v, o, s, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_backward(args, dist: Dist, pk):
     """Gradients of the 8K prefill (dq, dk, dv, ds0 for a given dO)."""
     import long_context_linear_b200 as la
@@ -681,6 +721,7 @@ def main():
         extras["decode_small_graph"] = run_decode_small_graph(args, dist, pk)
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
         extras["varlen"] = run_varlen(args, dist, pk)
+        extras["varlen_few_long"] = run_varlen_few(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
         extras["prefill_8k_d64"] = run_prefill8k(args, dist, pk, d=64)

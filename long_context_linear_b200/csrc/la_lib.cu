@@ -194,7 +194,8 @@ la_status after_launch(const char* what) {
 la_status launch_tc(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
     const bool general =
-        p.phi != LA_PHI_IDENTITY || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1);
+        p.phi != LA_PHI_IDENTITY || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1) ||
+        p.seg_off;
     auto go = [&](auto kern) { kern<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p); };
     if (p.dk == 64) general ? go(tc::prefill_tc_kernel<true, 64>) : go(tc::prefill_tc_kernel<false, 64>);
     else general ? go(tc::prefill_tc_kernel<true, 128>) : go(tc::prefill_tc_kernel<false, 128>);
@@ -463,16 +464,62 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc launch");
 }
 
+namespace {
+size_t varlen_order_bytes(int n_seq) { return n_seq > 0 ? round256((size_t)n_seq * sizeof(int)) : 0; }
+
+// Segment length (a multiple of C) for a packed batch whose (sequence, head,
+// slice) items fill less than half of the SMs, or 0 for no split.  The host
+// knows only the total token count T, so segments are sized for T spread over
+// about one item per SM.  LA_PREFILL_SEGMENTS = P forces about P segments per
+// sequence of average length (1: no split).
+int plan_varlen_segments(int n_seq, int T, int H, int d, int sms) {
+    if (n_seq <= 0 || T <= 0 || H <= 0) return 0;
+    const long C = tc::C;
+    if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
+        const int P = atoi(e);
+        if (P <= 1) return 0;
+        const long avg = ((long)T + n_seq - 1) / n_seq;
+        return (int)std::max(C, ((avg + P - 1) / P + C - 1) / C * C);
+    }
+    const long per_seq_items = (long)H * tc_slices(d);
+    if ((long)n_seq * per_seq_items * 2 > sms) return 0;
+    // at most S segments keep every item in one wave; rounding each sequence
+    // up to whole segments adds at most one per sequence, so size for S - n_seq
+    const long S = sms / per_seq_items;
+    if (S <= 2L * n_seq) return 0;
+    const long target = S - n_seq;
+    const long seg = std::max((long)kMinSegChunks * C, (((long)T + target - 1) / target + C - 1) / C * C);
+    return (long)T >= 2 * seg ? (int)seg : 0;
+}
+
+// Upper bounds of the segment counts (all segments / all but each sequence's
+// last) and the bytes of the segment area: the two offset arrays, the
+// segment sums and the segment starts.
+void varlen_segment_counts(int n_seq, int T, int seg_len, long* max_segs, long* max_nl) {
+    *max_nl = T / seg_len;
+    *max_segs = *max_nl + n_seq;
+}
+size_t varlen_segment_bytes(int n_seq, int T, int H, int d, int seg_len) {
+    long ms, mnl;
+    varlen_segment_counts(n_seq, T, seg_len, &ms, &mnl);
+    const size_t state = (size_t)H * d * d * sizeof(float);
+    return 2 * round256((size_t)(n_seq + 1) * sizeof(int)) + (size_t)mnl * state + (size_t)ms * state;
+}
+}  // namespace
+
 size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt) {
-    (void)T; (void)H; (void)dk; (void)dv; (void)dt;
-    if (n_seq <= 0) return 0;
-    return round256((size_t)n_seq * sizeof(int));
+    return la_prefill_varlen_workspace_size_ex(n_seq, T, H, dk, dv, dt, LA_PHI_IDENTITY);
 }
 
 size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int dv, la_dtype dt, la_phi phi) {
-    const size_t base = la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt);
+    const size_t base = varlen_order_bytes(n_seq);
     if (!base || T <= 0 || H <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return base;
-    return base + phi_workspace_bytes((long)T * H, dk, phi);
+    size_t total = base + phi_workspace_bytes((long)T * H, dk, phi);
+    DeviceInfo* di;
+    if (device_info(&di) != LA_OK) return total;
+    const int seg_len = plan_varlen_segments(n_seq, T, H, dk, di->sms);
+    if (seg_len) total += varlen_segment_bytes(n_seq, T, H, dk, seg_len);
+    return total;
 }
 
 la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
@@ -505,7 +552,7 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     if ((long)T * H > (1L << 40) || (long)n_seq * H > (1L << 30)) return fail(LA_ERR_INVALID_ARG, "problem too large");
     const bool tcpath = use_tensor_cores(dk, dt);
     if ((s = check_chunk(chunk, tcpath)) != LA_OK) return s;
-    const size_t need = la_prefill_varlen_workspace_size(n_seq, T, H, dk, dv, dt);
+    const size_t need = varlen_order_bytes(n_seq);
     if (tcpath && (ws_bytes < need || !workspace || !aligned16(workspace)))
         return fail(LA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu", need, ws_bytes);
     DeviceInfo* di;
@@ -543,12 +590,21 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
     if ((s = after_launch("varlen order launch")) != LA_OK) return s;
     const size_t ws_phi = T > 0 ? phi_workspace_bytes((long)T * H, dk, phi) : 0;
+    size_t off_seg = need;
     if (ws_phi && ws_bytes >= need + ws_phi) {
         if ((s = phi_prepass(&q, &k, reinterpret_cast<uint8_t*>(workspace) + need, (long)T * H * dk, phi, di, st)) !=
             LA_OK)
             return s;
         phi = LA_PHI_IDENTITY;
+        off_seg += ws_phi;
     }
+    const int nvs = tc_slices(dv);
+    int seg_len = plan_varlen_segments(n_seq, T, H, dk, di->sms);
+    long max_segs = 0, max_nl = 0;
+    if (seg_len) varlen_segment_counts(n_seq, T, seg_len, &max_segs, &max_nl);
+    if (seg_len && (ws_bytes < off_seg + varlen_segment_bytes(n_seq, T, H, dk, seg_len) ||
+                    max_segs * H * nvs > (1L << 30)))
+        seg_len = 0;  // no room for the segment states: whole sequences
 
     tc::Params p{};
     p.mode = 1;
@@ -573,6 +629,40 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     if ((s = make_map(&mk, k ? k : any, dk, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
     if ((s = make_map(&mv, v ? v : any, dv, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
     if ((s = make_map(&mo, o ? o : any, dv, H, Tm, head, tok, 1, 32)) != LA_OK) return s;
+    if (seg_len) {
+        // segments: offsets in work order, the sums of all but each sequence's
+        // last segment, the state before every segment, then every segment
+        uint8_t* w = reinterpret_cast<uint8_t*>(workspace) + off_seg;
+        const size_t ints = round256((size_t)(n_seq + 1) * sizeof(int));
+        int* seg_off = reinterpret_cast<int*>(w);
+        int* seg_off_nl = reinterpret_cast<int*>(w + ints);
+        float* sums = reinterpret_cast<float*>(w + 2 * ints);
+        float* starts = sums + (size_t)max_nl * H * dk * dv;
+        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, seg_len, seg_off, seg_off_nl);
+        if ((s = after_launch("varlen segment plan launch")) != LA_OK) return s;
+        p.seg_off = seg_off;
+        p.seg_off_nl = seg_off_nl;
+        p.n_seq = n_seq;
+        p.seg_len = seg_len;
+        if (max_nl > 0) {
+            tc::Params p1 = p;
+            p1.state_only = 1;
+            p1.n_items = (int)(max_nl * H * nvs);
+            p1.s_out = sums;
+            p1.pool = nullptr;
+            p1.init_idx = nullptr;
+            if ((s = launch_tc(std::min(p1.n_items, di->sms), mq, mk, mv, mo, p1, st,
+                               "prefill_tc (varlen segment sums) launch")) != LA_OK)
+                return s;
+        }
+        const long threads = (long)n_seq * H * (dk * dv / 4);
+        const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
+        segp::seg_prefix_varlen_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(sums, state_pool, init_idx, order, seg_off,
+                                                                            seg_off_nl, starts, n_seq, H, dk * dv);
+        if ((s = after_launch("varlen segment prefix launch")) != LA_OK) return s;
+        p.n_items = (int)(max_segs * H * nvs);
+        p.seg_init = starts;
+    }
     const int grid = std::min(p.n_items, di->sms);
     return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc (varlen) launch");
 }

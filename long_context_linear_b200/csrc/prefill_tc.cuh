@@ -119,6 +119,11 @@ struct Params {
     int init_transposed;   // the initial state is given as its transpose [dv][DK]
     int seg_base;          // dense: the items' segments are seg_base .. seg_base + n_seg - 1
     int dk;                // key dim = value dim: 128 or 64 (selects the kernel instance)
+    // packed only: segments of seg_len tokens (vorder::seg_plan_kernel offsets
+    // in work order over n_seq sequences), or null
+    const int* seg_off;
+    const int* seg_off_nl;
+    int n_seq;
 };
 
 struct Item {
@@ -168,6 +173,45 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
         it.init = p.seg_init ? p.seg_init + (long)us * KD * p.dv
                              : ((sg == first && p.s0) ? p.s0 + (long)u * KD * p.dv : nullptr);
         it.write_state = p.s_out_per_seg || sg == last;
+    } else if (kGeneral && p.seg_off) {
+        // packed batch cut into segments of seg_len tokens: item = (segment in
+        // work order, head, slice); the state-only pass numbers only the
+        // segments that are not a sequence's last.  Items past the device-side
+        // total (the host launches an upper bound) are empty.
+        const int* off = p.state_only ? p.seg_off_nl : p.seg_off;
+        const int hs = idx / NV;    // segment * H + head
+        const int sgi = hs / p.H;
+        const int h = hs - sgi * p.H;
+        it.c1 = h;
+        it.c2 = 0;
+        if (sgi >= off[p.n_seq]) {
+            it.t0 = 0;
+            it.len = 0;
+            it.state = 0;
+            it.init = nullptr;
+            it.write_state = false;
+        } else {
+            int lo = 0, hi = p.n_seq;  // rank r with off[r] <= sgi < off[r + 1]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (off[mid] <= sgi) lo = mid;
+                else hi = mid;
+            }
+            const int r = lo, sg = sgi - off[r];
+            const int seq = p.order[r];
+            const int end = p.cu_seqlens[seq + 1];
+            it.t0 = p.cu_seqlens[seq] + sg * p.seg_len;
+            it.len = max(0, min(p.seg_len, end - it.t0));
+            if (p.state_only) {
+                it.state = (long)sgi * p.H + h;  // index of this segment's sum
+                it.init = nullptr;
+                it.write_state = true;
+            } else {
+                it.state = (long)seq * p.H + h;
+                it.init = p.seg_init + ((long)sgi * p.H + h) * KD * p.dv;
+                it.write_state = sgi == off[r + 1] - 1;  // the sequence's last segment
+            }
+        }
     } else {
         const int hs = idx / NV;    // sequence rank * H + head
         const int r = hs / p.H;

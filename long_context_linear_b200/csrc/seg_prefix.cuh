@@ -56,5 +56,34 @@ seg_prefix_kernel(const float* __restrict__ seg_sums, const float* __restrict__ 
     }
 }
 
+// The same for a packed batch whose sequences have different segment counts
+// (seg_off, seg_off_nl from vorder::seg_plan_kernel, in work order): the state
+// before segment g of rank r, head h is pool[init_idx[seq]][h] (or zero) plus
+// the sums of the sequence's segments before g.
+//   seg_sums: [non-last segments][H][elems]   starts: [segments][H][elems]
+__global__ void __launch_bounds__(NUM_THREADS)
+seg_prefix_varlen_kernel(const float* __restrict__ seg_sums, const float* __restrict__ pool,
+                         const int* __restrict__ init_idx, const int* __restrict__ order, const int* __restrict__ seg_off,
+                         const int* __restrict__ seg_off_nl, float* __restrict__ starts, int n_seq, int H, int elems) {
+    const int per_unit = elems / 4;
+    const long total = (long)n_seq * H * per_unit;
+    for (long t = (long)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (long)gridDim.x * blockDim.x) {
+        const int r = static_cast<int>(t / ((long)H * per_unit));
+        const int rem = static_cast<int>(t - (long)r * H * per_unit);
+        const int h = rem / per_unit, e = (rem - h * per_unit) * 4;
+        const int sq = order[r];
+        const int ii = init_idx ? init_idx[sq] : -1;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (pool && ii >= 0) acc = *reinterpret_cast<const float4*>(pool + ((long)ii * H + h) * elems + e);
+        const int s0 = seg_off[r], cnt = seg_off[r + 1] - s0, nl0 = seg_off_nl[r];
+        *reinterpret_cast<float4*>(starts + ((long)s0 * H + h) * elems + e) = acc;
+        for (int g = 1; g < cnt; ++g) {
+            const float4 x = *reinterpret_cast<const float4*>(seg_sums + ((long)(nl0 + g - 1) * H + h) * elems + e);
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            *reinterpret_cast<float4*>(starts + ((long)(s0 + g) * H + h) * elems + e) = acc;
+        }
+    }
+}
+
 }  // namespace segp
 }  // namespace lcl

@@ -193,3 +193,18 @@ def test_varlen_phi_prepass_equals_in_kernel_mapping(la, phi):
     assert la.device_status() == 0
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_varlen_with_phi_and_segments(la, oracle_mod, monkeypatch, phi):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", "3")
+    lens = [2000, 1, 900]
+    cu = synth.cu_seqlens(lens)
+    T, H, d = int(cu[-1]), 2, 128
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=8)
+    o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.varlen(q, k, v, cu, phi=phi)
+    assert_out(o.cpu()[None], ro[None], torch.bfloat16, 1)
+    assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])

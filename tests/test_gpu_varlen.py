@@ -113,3 +113,48 @@ def test_varlen_many_short_sequences(la, oracle_mod, n_seq):
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
     assert_out(o[None], ro[None], torch.bfloat16, 1)
     assert_state(s, rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["2", "3", "7"])
+@pytest.mark.parametrize("d", [128, 64])
+def test_varlen_segments_match_oracle(la, oracle_mod, monkeypatch, segments, d):
+    """A packed batch cut into segments (LA_PREFILL_SEGMENTS forces about that
+    many per sequence of average length): the sums of all but each sequence's
+    last segment, per-sequence prefix states from the pool, then all segments.
+    Lengths include an empty sequence, a one-token one and ragged tails."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    lens = [1500, 0, 1, 700, 3000, 129]
+    cu, q, k, v, pool, idx = _case(lens, 3, d, "bf16", seed=61, n_pool=2, resume=[0, 1, -1, 1, -1, 0])
+    o, s = _run(la, cu, q, k, v, pool, idx)
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_state(s, rs, 2)
+
+
+def test_varlen_segments_automatic(la, oracle_mod):
+    """Two long sequences with two heads fill 8 of the SMs unsplit: the library
+    cuts them into segments by itself."""
+    lens = [9000, 5000]
+    cu, q, k, v, pool, idx = _case(lens, 2, 128, "bf16", seed=63, n_pool=1, resume=[0, -1])
+    assert la.prefill_varlen_workspace_size(2, sum(lens), 2, 128, torch.bfloat16) > 4 * 256
+    o, s = _run(la, cu, q, k, v, pool, idx)
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_state(s, rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["1", "4"])
+def test_varlen_segments_integer_inputs_bit_exact(la, oracle_mod, monkeypatch, segments):
+    """Inputs in {-1,0,1} with integer pool states: every partial sum is exact,
+    so the split and unsplit runs both equal the oracle bit for bit."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    lens = [1000, 3, 600, 0, 257]
+    cu = synth.cu_seqlens(lens)
+    T, H, d = int(cu[-1]), 2, 128
+    q, k, v = (synth.integer_valued((T, H, d), seed=s, dtype=torch.bfloat16) for s in (71, 72, 73))
+    pool = synth.integer_valued((2, H, d, d), seed=74, lo=-20, hi=20, dtype=torch.float32)
+    idx = torch.tensor([1, -1, 0, 0, -1], dtype=torch.int32)
+    o, s = _run(la, cu, q, k, v, pool, idx)
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    assert torch.equal(o, torch.from_numpy(ro).to(torch.bfloat16))
+    np.testing.assert_array_equal(to64(s), rs)
