@@ -46,12 +46,12 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 
 # DRAM traffic of one prefill launch, from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum) of the kernel built from sources with this hash, on
-# the H=16, N=32768 case: 517.80 MB for 16*32768 token-heads.  Traffic grows
+# the H=16, N=32768 case: 516.68 MB for 16*32768 token-heads.  Traffic grows
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "3c28761b61fecc54"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.98e6 + 113.45e6) / (16 * 32768)
+TRAFFIC_HASH = "6b18c8c19b5cf500"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.772224e6 + 113.908992e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
@@ -466,7 +466,8 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0):
     q, k, v = synth.dense(B, H, N, d, "bf16", seed=61 + dist.rank, device=dev)
     o = torch.empty_like(v)
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    # with phi != identity the workspace holds phi(q), phi(k) (mapped by a pre-pass)
+    # with elu + 1 the workspace holds phi(q), phi(k) (mapped by a pre-pass);
+    # relu is mapped on the tiles inside the prefill kernel
     ws_bytes = la.prefill_workspace_size(B, H, N, d, torch.bfloat16, phi)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -724,6 +725,7 @@ def main():
         extras["varlen_few_long"] = run_varlen_few(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk)
         extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
+        extras["prefill_8k_relu"] = run_prefill8k(args, dist, pk, "relu")
         extras["prefill_8k_d64"] = run_prefill8k(args, dist, pk, d=64)
         extras["few_heads"] = run_few_heads(args, dist, pk)
         extras["backward_8k"] = run_backward(args, dist, pk)

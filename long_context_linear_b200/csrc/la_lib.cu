@@ -104,10 +104,12 @@ la_status device_info(DeviceInfo** out) {
             return cuda_fail(e, "cudaDeviceGetAttribute");
         if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word)) != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress");
-        const void* tc_kernels[4] = {reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, 128>),
-                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, 128>),
-                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, 64>),
-                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, 64>)};
+        const void* tc_kernels[6] = {reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, false, 128>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, false, 128>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, true, 128>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<false, false, 64>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, false, 64>),
+                                     reinterpret_cast<const void*>(tc::prefill_tc_kernel<true, true, 64>)};
         for (const void* kern : tc_kernels)
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES)) !=
                 cudaSuccess)
@@ -189,16 +191,24 @@ la_status after_launch(const char* what) {
     return LA_OK;
 }
 
-// The tensor-core prefill for p.dk (128 or 64), lean instance unless an
-// option needs the general one.
+// The tensor-core prefill for p.dk (128 or 64): the lean instance unless an
+// option needs the general one, which carries the feature-map code only when
+// a feature map is applied in the kernel.
 la_status launch_tc(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
+    const bool phi = p.phi != LA_PHI_IDENTITY;
     const bool general =
-        p.phi != LA_PHI_IDENTITY || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1) ||
-        p.seg_off;
+        phi || p.reverse || p.state_only || p.init_transposed || (p.mode == 0 && p.n_seg > 1) || p.seg_off;
     auto go = [&](auto kern) { kern<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(mq, mk, mv, mo, p); };
-    if (p.dk == 64) general ? go(tc::prefill_tc_kernel<true, 64>) : go(tc::prefill_tc_kernel<false, 64>);
-    else general ? go(tc::prefill_tc_kernel<true, 128>) : go(tc::prefill_tc_kernel<false, 128>);
+    if (p.dk == 64) {
+        if (phi) go(tc::prefill_tc_kernel<true, true, 64>);
+        else if (general) go(tc::prefill_tc_kernel<true, false, 64>);
+        else go(tc::prefill_tc_kernel<false, false, 64>);
+    } else {
+        if (phi) go(tc::prefill_tc_kernel<true, true, 128>);
+        else if (general) go(tc::prefill_tc_kernel<true, false, 128>);
+        else go(tc::prefill_tc_kernel<false, false, 128>);
+    }
     return after_launch(what);
 }
 
@@ -315,9 +325,11 @@ size_t segment_workspace_bytes(long U, int P, int dk, int dv) {
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Scratch for phi(q) and phi(k) (bf16, `rows` rows of d) on the tensor-core
-// path; zero for the identity.
+// path, for elu + 1 only: its exponentials cost the prefill kernel more than a
+// separate bandwidth-bound pass over q and k, while relu (a packed max per
+// pair of values) is cheaper mapped on the tiles inside the kernel.
 size_t phi_workspace_bytes(long rows, int d, la_phi phi) {
-    if (phi == LA_PHI_IDENTITY || rows <= 0) return 0;
+    if (phi != LA_PHI_ELU1 || rows <= 0) return 0;
     return 2 * round256((size_t)rows * (size_t)d * 2);
 }
 

@@ -27,16 +27,27 @@ __device__ __forceinline__ float apply_phi_fast(float x, int phi) {
     return x;
 }
 
-// phi on 8 bf16 values packed in 16 bytes (fp32 evaluation, bf16 result to
-// nearest even).
+// phi on 8 bf16 values packed in 16 bytes, with the result of the fp32
+// evaluation above rounded to bf16 (nearest even), in packed bf16 pairs.
+// relu is one packed max per pair.  elu + 1 is written as
+// exp(min(x, 0)) + max(x, 0): for x <= 0 the bf16 exponential plus zero is
+// that exponential, and for x > 0 it is bf16(exp(0)) = 1 plus x, one
+// rounding of 1 + x, which is what rounding the fp32 sum gives as well
+// (1 + x is exact in fp32 for every bf16 x >= 2^-16, and rounds to 1 either
+// way below).
 __device__ __forceinline__ uint4 apply_phi_bf16x8(uint4 r, int phi) {
+    if (phi != PHI_ELU1 && phi != PHI_RELU) return r;
+    const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
     uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float lo = apply_phi_fast(__uint_as_float(w[i] << 16), phi);
-        const float hi = apply_phi_fast(__uint_as_float(w[i] & 0xffff0000u), phi);
-        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        __nv_bfloat162 y = __hmax2(x, zero);
+        if (phi == PHI_ELU1) {
+            const float2 m = __bfloat1622float2(__hmin2(x, zero));
+            y = __hadd2(__floats2bfloat162_rn(__expf(m.x), __expf(m.y)), y);
+        }
+        w[i] = *reinterpret_cast<const uint32_t*>(&y);
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }

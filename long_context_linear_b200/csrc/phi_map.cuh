@@ -2,10 +2,11 @@
 //
 // With a feature map other than the identity (page "MiniMax-M1で理解する…",
 // section "線形アテンションの数学的基礎": phi(Q) (phi(K)^T V)), the prefill reads
-// phi(Q) and phi(K) as tensor-core operands in bf16.  Mapping them in a
-// separate bandwidth-bound pass (read 2, write 2 arrays) costs less than
-// mapping the tiles in shared memory inside the pipelined kernel, where the
-// mapping sits on the chain that feeds the next chunk's product.  Both use
+// phi(Q) and phi(K) as tensor-core operands in bf16.  For elu + 1, mapping
+// them in a separate bandwidth-bound pass (read 2, write 2 arrays) costs less
+// than evaluating the exponentials on the tiles inside the pipelined kernel,
+// where the mapping sits on the chain that feeds the next chunk's product
+// (relu, one packed max per pair, is cheaper inside).  Both use
 // apply_phi_bf16x8, so the two routes give bit-identical operands.
 #pragma once
 #include "phi.cuh"

@@ -253,26 +253,28 @@ __device__ __noinline__ void clear_tail_rows(uint8_t* tile, int rows, int ksteps
     fence_proxy_async_smem();
 }
 
-// phi in place on 16-byte vectors [e0, e1) of a tile region, by the 128
-// state-warp threads (t = 0 .. 127); shared-memory addresses.  vec(e) maps a
-// vector index to its address.  Four vectors are loaded before any is
-// transformed.  Out of line: the identity path never runs it and should not
-// carry its code.
-__device__ __noinline__ void phi_region(uint32_t base, uint32_t panel_stride, int per_panel, int n, int t, int phi) {
+// phi in place on the 128 token rows of the NP 64-column panels of a Q or K
+// tile (panels `stride` bytes apart; the S^T rows behind K are left alone),
+// by the 128 state-warp threads t = 0 .. 127, in 16-byte vectors with four
+// loads in flight.  Only the feature-map instance carries this code.
+template <int NP>
+__device__ __forceinline__ void phi_tile(uint32_t base, uint32_t stride, int t, int phi) {
+    constexpr int PER_PANEL = PANEL / 16;
+    constexpr int PER_THREAD = NP * PER_PANEL / 128;
 #pragma unroll 1
-    for (int e0 = t; e0 < n; e0 += 4 * 128) {
+    for (int j0 = 0; j0 < PER_THREAD; j0 += 4) {
         uint32_t a[4];
         uint4 r[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int e = e0 + j * 128;
-            a[j] = base + static_cast<uint32_t>(e / per_panel) * panel_stride + static_cast<uint32_t>(e % per_panel) * 16u;
-            if (e < n) r[j] = ld_shared_v4(a[j]);
+            const int e = t + (j0 + j) * 128;
+            a[j] = base + static_cast<uint32_t>(e / PER_PANEL) * stride + static_cast<uint32_t>(e % PER_PANEL) * 16u;
+            r[j] = ld_shared_v4(a[j]);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint4 y = apply_phi_bf16x8(r[j], phi);
-            if (e0 + j * 128 < n) st_shared_v4(a[j], y.x, y.y, y.z, y.w);
+            st_shared_v4(a[j], y.x, y.y, y.z, y.w);
         }
     }
     fence_proxy_async_smem();
@@ -302,9 +304,11 @@ __device__ __forceinline__ constexpr uint64_t mnmaj_step(int kk) { return static
 // kGeneral = false is the lean instance for the common case (feature map
 // identity, chunks in order, outputs computed, initial state as given, whole
 // sequences): the options below are then compile-time constants and their
-// code is left out.  KD = d_k = d_v: 128 (two 64-column panels per Q and K
-// tile, two value slices per head) or 64 (one panel, one slice).
-template <bool kGeneral, int KD>
+// code is left out.  kPhi (with kGeneral) adds the feature map on Q and K
+// tiles; without it the general instance keeps the identity and stays
+// smaller.  KD = d_k = d_v: 128 (two 64-column panels per Q and K tile, two
+// value slices per head) or 64 (one panel, one slice).
+template <bool kGeneral, bool kPhi, int KD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -337,7 +341,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int G = gridDim.x;
     const int cta = blockIdx.x;
     const bool state_only = kGeneral && p.state_only;
-    const int phi = kGeneral ? p.phi : static_cast<int>(PHI_IDENTITY);
+    const int phi = kGeneral && kPhi ? p.phi : static_cast<int>(PHI_IDENTITY);
     const bool rev = kGeneral && p.reverse;
     const bool init_t = kGeneral && p.init_transposed;
     constexpr int NP = KD / 64;  // 64-column panels per Q / K tile
@@ -676,14 +680,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 }
                 if (phi != PHI_IDENTITY) {
                     // phi(K_c), then phi(Q_c), in place, before the tensor cores read
-                    // them (the S^T rows behind K are left alone); K first, so that
-                    // K^T V can start while Q is mapped
-                    phi_region(smem_u32(sm + OFF_K + ks * TILE_K), KPANEL, PANEL / 16, NP * PANEL / 16, i, phi);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&kphi_full[ks]);
-                    if (!state_only)
-                        phi_region(smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q), PANEL, PANEL / 16, NP * PANEL / 16, i,
-                                   phi);
+                    // them; K first, so that K^T V can start while Q is mapped
+#pragma unroll 1
+                    for (int reg = 0; reg < (state_only ? 1 : 2); ++reg) {
+                        phi_tile<NP>(reg == 0 ? smem_u32(sm + OFF_K + ks * TILE_K)
+                                              : smem_u32(sm + OFF_Q + (g % Q_SLOTS) * TILE_Q),
+                                     reg == 0 ? KPANEL : PANEL, i, phi);
+                        if (reg == 0) {
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&kphi_full[ks]);
+                        }
+                    }
                 }
                 if (!state_only) {
                     if (g >= 2 && !warp_wait(&o_empty[g & 1], ((g - 2) >> 1) & 1, abort, p.status)) { stop = true; break; }

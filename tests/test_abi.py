@@ -53,16 +53,17 @@ def test_workspace_sizes(lib):
 
 
 def test_workspace_sizes_with_feature_map(lib):
-    # identity adds nothing; elu+1 / relu add phi(q) and phi(k) in bf16 on the tensor-core path
-    assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, 0) == 0
-    for phi in (1, 2):
-        assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, phi) == 2 * 4 * 32 * 8192 * 128 * 2
-        assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 1, phi) == 0  # fp32: mapped at load
-        base = lib.la_prefill_varlen_workspace_size(64, 1000, 32, 128, 128, 0)
-        assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, phi) == base + 2 * 1000 * 32 * 256
-        assert lib.la_prefill_varlen_workspace_size_ex(64, 1001, 3, 128, 128, 0, phi) == base + 2 * (
-            (1001 * 3 * 256 + 255) // 256 * 256)
-    assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, 0) == base
+    # identity and relu (mapped inside the kernel) add nothing; elu+1 adds
+    # phi(q) and phi(k) in bf16 for the pre-pass on the tensor-core path
+    base = lib.la_prefill_varlen_workspace_size(64, 1000, 32, 128, 128, 0)
+    for phi in (0, 2):
+        assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, phi) == 0
+        assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, phi) == base
+    assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 0, 1) == 2 * 4 * 32 * 8192 * 128 * 2
+    assert lib.la_prefill_workspace_size_ex(4, 32, 8192, 128, 128, 1, 1) == 0  # fp32: mapped at load
+    assert lib.la_prefill_varlen_workspace_size_ex(64, 1000, 32, 128, 128, 0, 1) == base + 2 * 1000 * 32 * 256
+    assert lib.la_prefill_varlen_workspace_size_ex(64, 1001, 3, 128, 128, 0, 1) == (
+        lib.la_prefill_varlen_workspace_size(64, 1001, 3, 128, 128, 0) + 2 * ((1001 * 3 * 256 + 255) // 256 * 256))
 
 
 FAKE = 1 << 20  # a 16-byte aligned non-null "device pointer"; never dereferenced on these paths

@@ -149,14 +149,14 @@ def _raw_prefill(la, q, k, v, phi, ws):
     return o, s
 
 
-@pytest.mark.parametrize("phi", PHIS)
 @pytest.mark.parametrize("segments", [None, "3"])
-def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, phi, segments):
-    """With room in the workspace q and k are mapped by a pre-pass; without it
-    the kernel maps the tiles in shared memory.  Both round phi to bf16 the
-    same way, so the results are bit-identical."""
+def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, segments):
+    """With room in the workspace q and k are mapped by a pre-pass (elu + 1);
+    without it the kernel maps the tiles in shared memory.  Both round phi to
+    bf16 the same way, so the results are bit-identical."""
     if segments:
         monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    phi = "elu1"
     B, H, N = 1, 2, 3000
     q, k, v = synth.dense(B, H, N, 128, "bf16", seed=91, device="cuda")
     full = la.prefill_workspace_size(B, H, N, 128, torch.bfloat16, phi)
@@ -172,7 +172,15 @@ def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, phi, segments)
     assert torch.equal(s1, s2)
 
 
-@pytest.mark.parametrize("phi", PHIS)
+def test_relu_needs_no_phi_workspace(la):
+    """relu is mapped inside the prefill kernel whatever the workspace."""
+    assert la.prefill_workspace_size(2, 4, 3000, 128, torch.bfloat16, "relu") == \
+        la.prefill_workspace_size(2, 4, 3000, 128, torch.bfloat16)
+    assert la.prefill_varlen_workspace_size(3, 5000, 4, 128, torch.bfloat16, "relu") == \
+        la.prefill_varlen_workspace_size(3, 5000, 4, 128, torch.bfloat16)
+
+
+@pytest.mark.parametrize("phi", ["elu1"])
 def test_varlen_phi_prepass_equals_in_kernel_mapping(la, phi):
     lens = [700, 1, 129, 2000]
     cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
