@@ -150,7 +150,8 @@ def _raw_prefill(la, q, k, v, phi, ws):
 
 
 @pytest.mark.parametrize("segments", [None, "3"])
-def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, segments):
+@pytest.mark.parametrize("d", [128, 64])
+def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, segments, d):
     """With room in the workspace q and k are mapped by a pre-pass (elu + 1);
     without it the kernel maps the tiles in shared memory.  Both round phi to
     bf16 the same way, so the results are bit-identical."""
@@ -158,14 +159,31 @@ def test_tc_phi_prepass_equals_in_kernel_mapping(la, monkeypatch, segments):
         monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
     phi = "elu1"
     B, H, N = 1, 2, 3000
-    q, k, v = synth.dense(B, H, N, 128, "bf16", seed=91, device="cuda")
-    full = la.prefill_workspace_size(B, H, N, 128, torch.bfloat16, phi)
-    seg = la.prefill_workspace_size(B, H, N, 128, torch.bfloat16)
-    assert full >= seg + 2 * B * H * N * 128 * 2
+    q, k, v = synth.dense(B, H, N, d, "bf16", seed=91, device="cuda")
+    full = la.prefill_workspace_size(B, H, N, d, torch.bfloat16, phi)
+    seg = la.prefill_workspace_size(B, H, N, d, torch.bfloat16)
+    assert full >= seg + 2 * B * H * N * d * 2
     ws_full = torch.empty(full, dtype=torch.uint8, device="cuda")
     ws_seg = torch.empty(seg, dtype=torch.uint8, device="cuda") if seg else None
     o1, s1 = _raw_prefill(la, q, k, v, phi, ws_full)
     o2, s2 = _raw_prefill(la, q, k, v, phi, ws_seg)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    assert torch.equal(o1, o2)
+    assert torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("segments", [None, "3"])
+@pytest.mark.parametrize("d", [128, 64])
+def test_tc_relu_in_kernel_equals_identity_on_mapped_inputs(la, monkeypatch, segments, d):
+    """relu of a bf16 value is exact, so mapping the tiles inside the kernel
+    must give exactly the identity prefill of relu(q), relu(k) (mapped by
+    torch here)."""
+    if segments:
+        monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v = synth.dense(2, 3, 1500, d, "bf16", seed=93, device="cuda")
+    o1, s1 = la.prefill(q, k, v, phi="relu")
+    o2, s2 = la.prefill(torch.relu(q), torch.relu(k), v)
     torch.cuda.synchronize()
     assert la.device_status() == 0
     assert torch.equal(o1, o2)
