@@ -107,8 +107,8 @@ LA_API int la_version(void);
  *   workspace/ws_bytes: scratch of at least la_prefill_workspace_size(...)
  *          bytes, 16-byte aligned (may be NULL when that size is 0).  The size
  *          is non-zero when B*H units are too few to fill the GPU and N is
- *          long: the tensor-core path then cuts each sequence into segments of
- *          whole chunks (a segment split of the tiled form on page "MiniMax:
+ *          long: both paths (tensor cores and FFMA) then cut each sequence
+ *          into segments of whole chunks (a segment split of the tiled form on page "MiniMax:
  *          «Почему M2 в итоге стала моделью с полным вниманием?»", section 1,
  *          glossary entry "Lightning Attention": the K^T V sums of the
  *          segments give every segment its starting state).  The workspace

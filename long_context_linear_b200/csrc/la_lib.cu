@@ -293,13 +293,14 @@ int la_version(void) { return 200; }  // 0.2.0
 
 namespace {
 
-// Segment split of the dense tensor-core prefill: when the (unit, value slice)
-// items fill less than half of the SMs, each unit's sequence is cut into
-// segments of whole chunks (at least kMinSegChunks) so that about one item per
-// SM remains.  LA_PREFILL_SEGMENTS=<n> overrides the count (1 = no split).
+// Segment split of a dense prefill: when the items (one per unit and value
+// slice: d / 64 slices on the tensor cores, one on the FFMA path) fill less
+// than half of the SMs, each unit's sequence is cut into segments of whole
+// 128-token chunks (at least kMinSegChunks) so that about one item per SM
+// remains.  LA_PREFILL_SEGMENTS=<n> overrides the count (1 = no split).
 constexpr int kMinSegChunks = 8;
 
-int plan_segments(long U, int N, int d, int sms, int* seg_len) {
+int plan_segments(long U, int N, int slices, int sms, int* seg_len) {
     const int nch = (N + tc::C - 1) / tc::C;
     *seg_len = nch * tc::C;
     if (N <= 0) return 1;
@@ -307,7 +308,7 @@ int plan_segments(long U, int N, int d, int sms, int* seg_len) {
     if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
         P = atoi(e);
     } else {
-        const long items = U * (d / tc::DVS);
+        const long items = U * slices;
         P = items * 2 > sms ? 1 : (int)(sms / items);
         P = std::min(P, nch / kMinSegChunks);
     }
@@ -354,18 +355,70 @@ la_status phi_prepass(const void** q, const void** k, void* scratch, long elems,
 
 }  // namespace
 
+// The FFMA prefill over dense units.  When the units fill less than half of
+// the SMs and the workspace holds segment_workspace_bytes(U, P, d, d), each
+// unit's sequence is cut into P segments: a state-only pass sums K^T V per
+// segment (all but the last one visited), seg_prefix_kernel forms each
+// segment's starting state from them and `init`, and the main pass runs all
+// segments at once.  Otherwise one CTA runs each unit whole.
+la_status simt_dense(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
+                     float* s_out, bool reverse, la_phi phi, long U, int N, int d, la_dtype dt, int chunk,
+                     DeviceInfo* di, void* ws, size_t ws_bytes, cudaStream_t st) {
+    simt::Params sp{};
+    sp.mode = 0;
+    sp.N = N;
+    sp.s0 = init;
+    sp.s_out = s_out;
+    sp.phi = phi;
+    sp.reverse = reverse ? 1 : 0;
+    sp.init_transposed = init_t ? 1 : 0;
+    auto go = [&](const simt::Params& x, long grid) {
+        return dt == LA_FP32 ? launch_simt<float>(d, chunk, (int)grid, q, k, v, o, x, st)
+                             : launch_simt<__nv_bfloat16>(d, chunk, (int)grid, q, k, v, o, x, st);
+    };
+    int seg_len;
+    int P = plan_segments(U, N, 1, di->sms, &seg_len);
+    if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) || U * P > (1L << 30)))
+        P = 1;
+    if (P <= 1) return go(sp, U);
+    float* sums = reinterpret_cast<float*>(ws);
+    float* starts = sums + (size_t)U * (P - 1) * d * d;
+    simt::Params p1 = sp;
+    p1.n_seg = P - 1;
+    p1.seg_len = seg_len;
+    p1.seg_base = reverse ? 1 : 0;  // the segments whose sums reach another segment's start
+    p1.s0 = nullptr;
+    p1.init_transposed = 0;
+    p1.s_out = sums;
+    p1.s_out_per_seg = 1;
+    p1.state_only = 1;
+    la_status s;
+    if ((s = go(p1, U * (P - 1))) != LA_OK) return s;
+    const long threads = U * (long)(d * d / 4);
+    const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
+    segp::seg_prefix_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(sums, init, starts, U, P, d * d, reverse ? 1 : 0,
+                                                                 init_t ? 1 : 0, d);
+    if ((s = after_launch("segment prefix launch")) != LA_OK) return s;
+    sp.n_seg = P;
+    sp.seg_len = seg_len;
+    sp.seg_init = starts;
+    return go(sp, U * P);
+}
+
 size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt) {
     return la_prefill_workspace_size_ex(B, H, N, dk, dv, dt, LA_PHI_IDENTITY);
 }
 
 size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtype dt, la_phi phi) {
-    if (B <= 0 || H <= 0 || N <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return 0;
+    if (B <= 0 || H <= 0 || N <= 0 || dk != dv || (dk != 64 && dk != 128)) return 0;
+    const bool tc = use_tensor_cores(dk, dt);
     const long U = (long)B * H;
-    const size_t ph = phi_workspace_bytes(U * N, dk, phi);
+    const size_t ph = tc ? phi_workspace_bytes(U * N, dk, phi) : 0;
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return ph;
     int seg_len;
-    const size_t seg = segment_workspace_bytes(U, plan_segments(U, N, dk, di->sms, &seg_len), dk, dv);
+    const int P = plan_segments(U, N, tc ? tc_slices(dk) : 1, di->sms, &seg_len);
+    const size_t seg = segment_workspace_bytes(U, P, dk, dv);
     return ph ? round256(seg) + ph : seg;
 }
 
@@ -396,12 +449,8 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-    if (!tcpath) {
-        simt::Params sp{};
-        sp.mode = 0; sp.N = N; sp.s0 = s0; sp.s_out = s_out; sp.phi = phi;
-        if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)U, q, k, v, o, sp, st);
-        return launch_simt<__nv_bfloat16>(dk, chunk, (int)U, q, k, v, o, sp, st);
-    }
+    if (!tcpath)
+        return simt_dense(q, k, v, o, s0, false, s_out, false, phi, U, N, dk, dt, chunk, di, workspace, ws_bytes, st);
 
     const int nvs = tc_slices(dv);
     tc::Params p{};
@@ -419,7 +468,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     p.phi = phi;
     if (N == 0 && !s_out) return LA_OK;
     int seg_len;
-    int P = plan_segments(U, N, dk, di->sms, &seg_len);
+    int P = plan_segments(U, N, tc_slices(dk), di->sms, &seg_len);
     p.seg_len = seg_len;
     const size_t ws_need = segment_workspace_bytes(U, P, dk, dv);
     if (P > 1 && (!workspace || ws_bytes < ws_need || !aligned16(workspace) ||
@@ -852,7 +901,7 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     p.reverse = reverse ? 1 : 0;
     p.init_transposed = init_t ? 1 : 0;
     int seg_len;
-    int P = plan_segments(U, N, d, di->sms, &seg_len);
+    int P = plan_segments(U, N, tc_slices(d), di->sms, &seg_len);
     if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) ||
                   U * P * nvs > (1L << 30)))
         P = 1;
@@ -893,29 +942,14 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     return launch_tc(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_tc (backward pass) launch");
 }
 
-// The same on the FFMA path (fp32 inputs, or d = 64).
-static la_status simt_dense_pass(const void* q, const void* k, const void* v, void* o, const float* init, bool init_t,
-                          float* s_out, bool reverse, long U, int N, int d, la_dtype dt, cudaStream_t st) {
-    if (N == 0 && !s_out) return LA_OK;
-    simt::Params sp{};
-    sp.mode = 0;
-    sp.N = N;
-    sp.s0 = init;
-    sp.s_out = s_out;
-    sp.phi = LA_PHI_IDENTITY;
-    sp.reverse = reverse ? 1 : 0;
-    sp.init_transposed = init_t ? 1 : 0;
-    if (dt == LA_FP32) return launch_simt<float>(d, 0, (int)U, q, k, v, o, sp, st);
-    return launch_simt<__nv_bfloat16>(d, 0, (int)U, q, k, v, o, sp, st);
-}
-
 size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v, la_dtype dt) {
-    if (B <= 0 || H <= 0 || N <= 0 || !use_tensor_cores(d_k, dt) || d_k != d_v) return 0;
+    if (B <= 0 || H <= 0 || N <= 0 || d_k != d_v || (d_k != 64 && d_k != 128)) return 0;
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return 0;
     int seg_len;
     const long U = (long)B * H;
-    return segment_workspace_bytes(U, plan_segments(U, N, d_k, di->sms, &seg_len), d_k, d_v);
+    const int slices = use_tensor_cores(d_k, dt) ? tc_slices(d_k) : 1;
+    return segment_workspace_bytes(U, plan_segments(U, N, slices, di->sms, &seg_len), d_k, d_v);
 }
 
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,
@@ -964,11 +998,17 @@ la_status la_prefill_backward_ex(const void* q, const void* k, const void* v, co
         // (the passes run in stream order, so they share the workspace)
         return tc_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, di, st, workspace, ws_bytes);
     }
+    if (N == 0 && !ds0) return LA_OK;
     if (N > 0) {
-        if ((s = simt_dense_pass(dout, v, k, dq, s0, true, nullptr, false, U, N, d_k, dt, st)) != LA_OK) return s;
-        if ((s = simt_dense_pass(v, dout, q, dk, ds_n, true, nullptr, true, U, N, d_k, dt, st)) != LA_OK) return s;
+        if ((s = simt_dense(dout, v, k, dq, s0, true, nullptr, false, LA_PHI_IDENTITY, U, N, d_k, dt, 0, di,
+                            workspace, ws_bytes, st)) != LA_OK)
+            return s;
+        if ((s = simt_dense(v, dout, q, dk, ds_n, true, nullptr, true, LA_PHI_IDENTITY, U, N, d_k, dt, 0, di,
+                            workspace, ws_bytes, st)) != LA_OK)
+            return s;
     }
-    return simt_dense_pass(k, q, dout, dv, ds_n, false, ds0, true, U, N, d_k, dt, st);
+    return simt_dense(k, q, dout, dv, ds_n, false, ds0, true, LA_PHI_IDENTITY, U, N, d_k, dt, 0, di, workspace,
+                      ws_bytes, st);
 }
 
 size_t la_prefill_host_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt, int group) {

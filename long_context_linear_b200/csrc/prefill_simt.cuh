@@ -1,14 +1,16 @@
 // Chunked causal linear attention on CUDA cores (FFMA, fp32 throughout).
 //
 // Serves fp32 inputs (where the state must stay within ~1e-4 of the exact
-// result, beyond what bf16 tensor-core operands give) and d = 64.  Same tiled
+// result, beyond what bf16 tensor-core operands give).  Same tiled
 // form as the tensor-core path (page "MiniMax: «Почему M2 в итоге стала моделью
 // с полным вниманием?» (конспект)", section 1, glossary entry "Lightning
 // Attention"), with chunks of CS tokens:
 //   A   = (Q_c K_c^T) ⊙ M        M keeps s <= t
 //   O_c = A V_c + Q_c S
 //   S  += K_c^T V_c
-// One CTA per (unit | sequence, head), 256 threads.  Every product is
+// One CTA per (unit | segment of a unit | sequence, head), 256 threads; a
+// segment starts from a given state, and a state-only launch sums K^T V over
+// its segments without reading Q or writing outputs.  Every product is
 // register-tiled (each thread owns a block of outputs and reads 16-byte
 // vectors from shared memory), tiles wholly above the causal diagonal are
 // skipped, the state S stays in the registers of its owner threads between
@@ -38,6 +40,15 @@ struct Params {
     // chunk, so that o_t = q_t (S_init + sum_{s >= t} k_s v_s^T)
     int reverse;
     int init_transposed;    // the initial state is given as its transpose [d][d]
+    // dense only: each unit's sequence cut into segments of seg_len tokens; a
+    // launch covers segments seg_base .. seg_base + n_seg - 1 of every unit
+    // (CTA = unit * n_seg + j); n_seg = 0 means whole sequences
+    int n_seg;
+    int seg_len;
+    int seg_base;
+    const float* seg_init;  // [U][n_seg][d][d]: state before each segment, or null
+    int s_out_per_seg;      // 1: s_out is [U][n_seg][d][d], one state per segment
+    int state_only;         // 1: only S = (init) + sum K^T V over the segment
 };
 
 // Shared-memory layout (floats), rows padded by 4 so that 16-byte vectors
@@ -161,8 +172,26 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 
     long row0, row_stride, state;
     int len;
+    bool write_state = true;
+    bool init_t = p.init_transposed;
     const float* init = nullptr;
-    if (p.mode == 0) {
+    if (p.mode == 0 && p.n_seg > 0) {
+        // segment seg of unit u: tokens seg * seg_len .. (the last one may be shorter)
+        const int u = blockIdx.x / p.n_seg, j = blockIdx.x % p.n_seg, seg = p.seg_base + j;
+        const int t0 = seg * p.seg_len, n_all = (p.N + p.seg_len - 1) / p.seg_len;
+        row0 = (long)u * p.N + t0;
+        row_stride = 1;
+        len = min(p.seg_len, p.N - t0);
+        state = p.s_out_per_seg ? (long)u * p.n_seg + j : u;
+        // without one state per segment only the segment visited last writes S
+        write_state = p.s_out_per_seg || (p.reverse ? seg == 0 : seg == n_all - 1);
+        if (p.seg_init) {
+            init = p.seg_init + ((long)u * p.n_seg + j) * D * D;
+            init_t = false;
+        } else if (p.s0) {
+            init = p.s0 + (long)u * D * D;
+        }
+    } else if (p.mode == 0) {
         const int u = blockIdx.x;
         row0 = (long)u * p.N;
         row_stride = 1;
@@ -187,12 +216,13 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 #pragma unroll
         for (int c = 0; c < TN3; ++c) {
             const int j = col_of<TN3, D>(tx, c);
-            accS[r][c] = init ? init[p.init_transposed ? j * D + i : i * D + j] : 0.f;
+            accS[r][c] = init ? init[init_t ? j * D + i : i * D + j] : 0.f;
         }
         st_cols<TN3, D>(Sm + i * LV, tx, accS[r]);
     }
 
     const bool rev = p.reverse;
+    const bool state_only = p.state_only;
     const int nc = (len + CS - 1) / CS;
     for (int ci = 0; ci < nc; ++ci) {
         const int c0 = (rev ? nc - 1 - ci : ci) * CS;
@@ -203,7 +233,8 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             constexpr int LINES = D * (int)sizeof(T) / 128;
             const int n0 = (rev ? nc - 2 - ci : ci + 1) * CS;
             const int nrows = min(CS, len - n0);
-            for (int f = tid; f < 3 * nrows * LINES; f += NUM_THREADS) {
+            const int first = state_only ? 1 : 0;  // q is not read for the state alone
+            for (int f = tid + first * nrows * LINES; f < 3 * nrows * LINES; f += NUM_THREADS) {
                 const int which = f / (nrows * LINES), rl = f % (nrows * LINES);
                 const long g = (row0 + (long)(n0 + rl / LINES) * row_stride) * D;
                 const T* src = which == 0 ? q : (which == 1 ? k : v);
@@ -215,7 +246,12 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             float qv[VEC], kv[VEC], vv[VEC];
             if (t < rows) {
                 const long g = (row0 + (long)(c0 + t) * row_stride) * D + cc;
-                unpack16(*reinterpret_cast<const uint4*>(q + g), qv);
+                if (!state_only) {
+                    unpack16(*reinterpret_cast<const uint4*>(q + g), qv);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) qv[e] = 0.f;
+                }
                 unpack16(*reinterpret_cast<const uint4*>(k + g), kv);
                 unpack16(*reinterpret_cast<const uint4*>(v + g), vv);
 #pragma unroll
@@ -238,7 +274,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         }
         __syncthreads();
         // ---- scores: At[s][t] = q_t . k_s for s <= t (s >= t in reverse), else 0
-        {
+        if (!state_only) {
             const int t0 = ty * TM1, s0 = tx * TN1;
             float acc[TM1][TN1];
 #pragma unroll
@@ -267,7 +303,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         }
         __syncthreads();
         // ---- outputs: O_t = sum_s At[s][t] v_s + q_t S (s <= t, or s >= t in reverse)
-        {
+        if (!state_only) {
             const int t0 = ty * TM2;
             float acc[TM2][TN2];
 #pragma unroll
@@ -323,7 +359,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 #pragma unroll
         for (int r = 0; r < TM3; ++r) st_cols<TN3, D>(Sm + (ty * TM3 + r) * LV, tx, accS[r]);
     }
-    if (p.s_out) {
+    if (p.s_out && write_state) {
         float* dst = p.s_out + state * D * D;
 #pragma unroll
         for (int r = 0; r < TM3; ++r) {

@@ -149,3 +149,33 @@ def test_backward_tc_segments_integer_inputs_bit_exact(la, oracle_mod, monkeypat
     for g, r in ((dq, rq), (dk, rk), (dv, rv)):
         assert torch.equal(g.cpu(), torch.from_numpy(r).to(torch.bfloat16))
     np.testing.assert_array_equal(to64(ds0.cpu()), rs0)
+
+
+@pytest.mark.parametrize("segments,d", [("2", 128), ("3", 128), ("3", 64)])
+def test_backward_ffma_segments_match_oracle(la, oracle_mod, monkeypatch, segments, d):
+    """fp32: each FFMA pass cut into segments (state-only pass, prefix or, in
+    reverse order, suffix over the segment sums, then all segments)."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v, dout, s0, ds_n = _grad_case(1, 2, 3000, d, "fp32", seed=33, with_states=True)
+    dq, dk, dv, ds0 = la.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), s0.cuda(), ds_n.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
+    for g, r in ((dq, rq), (dk, rk), (dv, rv)):
+        _check(g.cpu(), r, q.dtype)
+    assert_state(ds0.cpu(), rs0, 2, tol=1e-4)
+
+
+@pytest.mark.parametrize("segments", ["2", "5"])
+def test_backward_ffma_segments_integer_bit_exact(la, oracle_mod, monkeypatch, segments):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N, d = 1, 2, 1300, 128
+    q, k, v, dout = (synth.integer_valued((B, H, N, d), seed=s) for s in (71, 72, 73, 74))
+    s0 = synth.integer_valued((B, H, d, d), seed=75, lo=-20, hi=20)
+    ds_n = synth.integer_valued((B, H, d, d), seed=76, lo=-20, hi=20)
+    dq, dk, dv, ds0 = la.prefill_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), s0.cuda(), ds_n.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    rq, rk, rv, rs0 = oracle_mod.backward(q, k, v, dout, s0, ds_n)
+    for g, r in ((dq, rq), (dk, rk), (dv, rv), (ds0, rs0)):
+        np.testing.assert_array_equal(to64(g.cpu()), r)

@@ -119,3 +119,67 @@ def test_segments_d64(la, oracle_mod, monkeypatch, segments):
     ro, rs = oracle_mod.recurrent(q, k, v, s0)
     assert_out(o, ro, torch.bfloat16, 2)
     assert_state(s, rs, 2)
+
+
+# ---------------------------------------------------------------- FFMA path
+# fp32 inputs run on the FFMA prefill, one CTA per (unit, segment); the same
+# split applies when the units fill less than half of the SMs.
+
+@pytest.mark.parametrize("B,H,N", [(1, 1, 9000), (1, 2, 5000 + 77)])
+@pytest.mark.parametrize("d", [128, 64])
+def test_ffma_auto_segments_match_oracle(la, oracle_mod, B, H, N, d):
+    assert la.prefill_workspace_size(B, H, N, d, torch.float32) > 0, "shape should be split"
+    q, k, v = synth.dense(B, H, N, d, "fp32", seed=3 * N + d)
+    s0 = _state(B, H, d, seed=N + 1)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.float32, 2)
+    assert_state(s, rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["2", "3", "7"])
+@pytest.mark.parametrize("chunk", [0, 32])
+def test_ffma_forced_segments(la, oracle_mod, monkeypatch, segments, chunk):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    q, k, v = synth.dense(1, 2, 3000, 128, "fp32", seed=41)
+    s0 = _state(1, 2, 128, seed=42)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), s0.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o.cpu(), ro, torch.float32, 2)
+    assert_state(s.cpu(), rs, 2)
+
+
+@pytest.mark.parametrize("segments", ["1", "4", "9"])
+@pytest.mark.parametrize("d", [128, 64])
+def test_ffma_segments_integer_inputs_bit_exact(la, oracle_mod, monkeypatch, segments, d):
+    """Inputs in {-1,0,1} and an integer S0 keep every fp32 product and partial
+    sum exact, so the split must not change a single bit."""
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N = 1, 2, 1500
+    q, k, v = (synth.integer_valued((B, H, N, d), seed=s) for s in (51, 52, 53))
+    s0 = synth.integer_valued((B, H, d, d), seed=54, lo=-20, hi=20)
+    o, s = _run(la, q, k, v, s0)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    np.testing.assert_array_equal(to64(o), ro)
+    np.testing.assert_array_equal(to64(s), rs)
+
+
+@pytest.mark.parametrize("phi", ["elu1", "relu"])
+def test_ffma_segments_with_phi(la, oracle_mod, monkeypatch, phi):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", "3")
+    q, k, v = synth.dense(1, 2, 2500, 128, "fp32", seed=61)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, phi=phi)
+    assert_out(o.cpu(), ro, torch.float32, 2)
+    assert_state(s.cpu(), rs, 2)
+
+
+def test_ffma_workspace_size_follows_the_plan(la):
+    # one item per unit on the FFMA path: 128 units fill the GPU, 8 do not
+    assert la.prefill_workspace_size(1, 128, 65536, 128, torch.float32) == 0
+    n = la.prefill_workspace_size(1, 8, 65536, 128, torch.float32)
+    assert n > 0 and n % (8 * 128 * 128 * 4) == 0
