@@ -256,7 +256,8 @@ LA_API la_status la_prefill_host(const void* q, const void* k, const void* v, vo
  * (dq = prefill(dout, v, k) from s0^T; dk = prefill(v, dout, q) from ds_n^T
  * and dv = prefill(k, q, dout) from ds_n, both with time reversed), with the
  * prefill's precision.  fp32: the same three passes on the FFMA
- * prefill kernel, fp32 arithmetic.
+ * prefill kernel, fp32 arithmetic.  LA_BACKWARD_SIMT=1 in the environment
+ * sends bf16 to the FFMA passes too (for testing).
  * d_k = d_v in {64, 128}.  All pointers 16-byte aligned; the caller owns every
  * buffer; no host synchronisation.  Errors: LA_ERR_INVALID_ARG (null, negative,
  * misaligned), LA_ERR_UNSUPPORTED (dims), LA_ERR_CUDA (launch).
@@ -268,9 +269,10 @@ LA_API la_status la_prefill_backward(const void* q, const void* k, const void* v
                                      la_stream_t stream);
 /* la_prefill_backward with a workspace (device, 16-byte aligned) of at least
  * la_prefill_backward_workspace_size(...) bytes: when the (batch, head) units
- * fill less than half of the SMs, each tensor-core pass cuts the sequences
- * into segments as la_prefill does (in reverse order the segment starts are
- * suffix sums).  With a smaller workspace (or none) the passes run unsplit. */
+ * fill less than half of the SMs, each pass (tensor-core or FFMA) cuts the
+ * sequences into segments as la_prefill does (in reverse order the segment
+ * starts are suffix sums).  With a smaller workspace (or none) the passes run
+ * unsplit. */
 LA_API size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v, la_dtype dt);
 LA_API la_status la_prefill_backward_ex(const void* q, const void* k, const void* v, const void* dout,
                                         const float* s0, const float* ds_n, void* dq, void* dk, void* dv, float* ds0,
