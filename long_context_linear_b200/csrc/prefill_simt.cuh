@@ -54,13 +54,15 @@ struct Params {
 // Shared-memory layout (floats), rows padded by 4 so that 16-byte vectors
 // stay aligned and successive rows start in different banks:
 //   Qt, Kt [D][CS+4]   Q and K transposed (token index contiguous)
-//   Vn     [CS][D+4]   V as stored
+//   Kn, Vn [CS][D+4]   K and V as stored (K twice: the scores read it by key
+//                      dimension, the state update by token)
 //   At     [CS][CS+4]  masked scores, transposed: At[s][t] = (q_t . k_s) [s <= t]
 //   Sm     [D][D+4]    the state before this chunk
 template <int D, int CS>
 constexpr int smem_bytes() {
-    return (2 * D * (CS + 4) + CS * (D + 4) + CS * (CS + 4) + D * (D + 4)) * 4;
+    return (2 * D * (CS + 4) + 2 * CS * (D + 4) + CS * (CS + 4) + D * (D + 4)) * 4;
 }
+static_assert(smem_bytes<128, 64>() <= 232448, "exceeds the 227 KB per-block shared memory limit");
 
 // Register tiles: the 256 threads form a 16 x 16 grid (ty = tid / 16 picks
 // the tile row, tx = tid % 16 the tile column); each thread owns TM x TN
@@ -165,7 +167,8 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
     extern __shared__ float sf[];
     float* Qt = sf;
     float* Kt = Qt + D * LQ;
-    float* Vn = Kt + D * LQ;
+    float* Kn = Kt + D * LQ;
+    float* Vn = Kn + CS * LV;
     float* At = Vn + CS * LV;
     float* Sm = At + CS * LQ;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -269,8 +272,10 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                 Kt[(cc + e) * LQ + t] = kv[e];
             }
 #pragma unroll
-            for (int e = 0; e < VEC; e += 4)
+            for (int e = 0; e < VEC; e += 4) {
+                *reinterpret_cast<float4*>(Kn + t * LV + cc + e) = make_float4(kv[e], kv[e + 1], kv[e + 2], kv[e + 3]);
                 *reinterpret_cast<float4*>(Vn + t * LV + cc + e) = make_float4(vv[e], vv[e + 1], vv[e + 2], vv[e + 3]);
+            }
         }
         __syncthreads();
         // ---- scores: At[s][t] = q_t . k_s for s <= t (s >= t in reverse), else 0
@@ -348,8 +353,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 #pragma unroll 2
         for (int s = 0; s < rows; ++s) {
             float a[TM3], b[TN3];
-#pragma unroll
-            for (int r = 0; r < TM3; ++r) a[r] = Kt[(ty * TM3 + r) * LQ + s];
+            ld_run<TM3>(Kn + s * LV + ty * TM3, a);
             ld_cols<TN3, D>(Vn + s * LV, tx, b);
 #pragma unroll
             for (int r = 0; r < TM3; ++r)
