@@ -529,11 +529,12 @@ namespace {
 size_t varlen_order_bytes(int n_seq) { return n_seq > 0 ? round256((size_t)n_seq * sizeof(int)) : 0; }
 
 // Segment length (a multiple of C) for a packed batch whose (sequence, head,
-// slice) items fill less than half of the SMs, or 0 for no split.  The host
+// value slice) items fill less than half of the SMs (`slices` per sequence and
+// head: d / 64 on the tensor cores, 1 on the FFMA path), or 0 for no split.  The host
 // knows only the total token count T, so segments are sized for T spread over
 // about one item per SM.  LA_PREFILL_SEGMENTS = P forces about P segments per
 // sequence of average length (1: no split).
-int plan_varlen_segments(int n_seq, int T, int H, int d, int sms) {
+int plan_varlen_segments(int n_seq, int T, int H, int slices, int sms) {
     if (n_seq <= 0 || T <= 0 || H <= 0) return 0;
     const long C = tc::C;
     if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
@@ -542,7 +543,7 @@ int plan_varlen_segments(int n_seq, int T, int H, int d, int sms) {
         const long avg = ((long)T + n_seq - 1) / n_seq;
         return (int)std::max(C, ((avg + P - 1) / P + C - 1) / C * C);
     }
-    const long per_seq_items = (long)H * tc_slices(d);
+    const long per_seq_items = (long)H * slices;
     if ((long)n_seq * per_seq_items * 2 > sms) return 0;
     // at most S segments keep every item in one wave; rounding each sequence
     // up to whole segments adds at most one per sequence, so size for S - n_seq
@@ -574,11 +575,12 @@ size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv,
 
 size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int dv, la_dtype dt, la_phi phi) {
     const size_t base = varlen_order_bytes(n_seq);
-    if (!base || T <= 0 || H <= 0 || !use_tensor_cores(dk, dt) || dk != dv) return base;
-    size_t total = base + phi_workspace_bytes((long)T * H, dk, phi);
+    if (!base || T <= 0 || H <= 0 || dk != dv || (dk != 64 && dk != 128)) return base;
+    const bool tc = use_tensor_cores(dk, dt);
+    size_t total = base + (tc ? phi_workspace_bytes((long)T * H, dk, phi) : 0);
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return total;
-    const int seg_len = plan_varlen_segments(n_seq, T, H, dk, di->sms);
+    const int seg_len = plan_varlen_segments(n_seq, T, H, tc ? tc_slices(dk) : 1, di->sms);
     if (seg_len) total += varlen_segment_bytes(n_seq, T, H, dk, seg_len);
     return total;
 }
@@ -642,9 +644,49 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         simt::Params sp{};
         sp.mode = 1; sp.H = H; sp.cu_seqlens = cu_seqlens; sp.pool = state_pool; sp.init_idx = init_idx;
         sp.s_out = s_out; sp.phi = phi;
-        const long grid = (long)n_seq * H;
-        if (dt == LA_FP32) return launch_simt<float>(dk, chunk, (int)grid, q, k, v, o, sp, st);
-        return launch_simt<__nv_bfloat16>(dk, chunk, (int)grid, q, k, v, o, sp, st);
+        auto go = [&](const simt::Params& x, long grid) {
+            return dt == LA_FP32 ? launch_simt<float>(dk, chunk, (int)grid, q, k, v, o, x, st)
+                                 : launch_simt<__nv_bfloat16>(dk, chunk, (int)grid, q, k, v, o, x, st);
+        };
+        // the segment split as on the tensor cores (one item per sequence and
+        // head), when the workspace has room for the order and the segment area
+        const int seg_len = plan_varlen_segments(n_seq, T, H, 1, di->sms);
+        long max_segs = 0, max_nl = 0;
+        if (seg_len) varlen_segment_counts(n_seq, T, seg_len, &max_segs, &max_nl);
+        if (!seg_len || !workspace || !aligned16(workspace) || max_segs * H > (1L << 30) ||
+            ws_bytes < need + varlen_segment_bytes(n_seq, T, H, dk, seg_len))
+            return go(sp, (long)n_seq * H);
+        int* order = reinterpret_cast<int*>(workspace);
+        vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
+        if ((s = after_launch("varlen order launch")) != LA_OK) return s;
+        uint8_t* w = reinterpret_cast<uint8_t*>(workspace) + need;
+        const size_t ints = round256((size_t)(n_seq + 1) * sizeof(int));
+        int* seg_off = reinterpret_cast<int*>(w);
+        int* seg_off_nl = reinterpret_cast<int*>(w + ints);
+        float* sums = reinterpret_cast<float*>(w + 2 * ints);
+        float* starts = sums + (size_t)max_nl * H * dk * dv;
+        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, seg_len, seg_off, seg_off_nl);
+        if ((s = after_launch("varlen segment plan launch")) != LA_OK) return s;
+        sp.order = order;
+        sp.seg_off = seg_off;
+        sp.seg_off_nl = seg_off_nl;
+        sp.n_seq = n_seq;
+        sp.seg_len = seg_len;
+        if (max_nl > 0) {
+            simt::Params p1 = sp;
+            p1.state_only = 1;
+            p1.s_out = sums;
+            p1.pool = nullptr;
+            p1.init_idx = nullptr;
+            if ((s = go(p1, max_nl * H)) != LA_OK) return s;
+        }
+        const long threads = (long)n_seq * H * (dk * dv / 4);
+        const int blocks = (int)std::min<long>((threads + segp::NUM_THREADS - 1) / segp::NUM_THREADS, 4L * di->sms);
+        segp::seg_prefix_varlen_kernel<<<blocks, segp::NUM_THREADS, 0, st>>>(sums, state_pool, init_idx, order, seg_off,
+                                                                            seg_off_nl, starts, n_seq, H, dk * dv);
+        if ((s = after_launch("varlen segment prefix launch")) != LA_OK) return s;
+        sp.seg_init = starts;
+        return go(sp, max_segs * H);
     }
 
     int* order = reinterpret_cast<int*>(workspace);
@@ -660,7 +702,7 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         off_seg += ws_phi;
     }
     const int nvs = tc_slices(dv);
-    int seg_len = plan_varlen_segments(n_seq, T, H, dk, di->sms);
+    int seg_len = plan_varlen_segments(n_seq, T, H, nvs, di->sms);
     long max_segs = 0, max_nl = 0;
     if (seg_len) varlen_segment_counts(n_seq, T, seg_len, &max_segs, &max_nl);
     if (seg_len && (ws_bytes < off_seg + varlen_segment_bytes(n_seq, T, H, dk, seg_len) ||

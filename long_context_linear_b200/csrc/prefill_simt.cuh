@@ -49,6 +49,15 @@ struct Params {
     const float* seg_init;  // [U][n_seg][d][d]: state before each segment, or null
     int s_out_per_seg;      // 1: s_out is [U][n_seg][d][d], one state per segment
     int state_only;         // 1: only S = (init) + sum K^T V over the segment
+    // packed only: segments of seg_len tokens, CTA = segment * H + head, with
+    // the segments numbered in the work order of `order` (vorder::
+    // seg_plan_kernel offsets over n_seq sequences); a state-only launch numbers
+    // only the segments that are not a sequence's last (seg_off_nl).  CTAs past
+    // the device-side total (the host launches an upper bound) do nothing.
+    const int* order;
+    const int* seg_off;
+    const int* seg_off_nl;
+    int n_seq;
 };
 
 // Shared-memory layout (floats), rows padded by 4 so that 16-byte vectors
@@ -201,6 +210,29 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         len = p.N;
         state = u;
         if (p.s0) init = p.s0 + (long)u * D * D;
+    } else if (p.seg_off) {
+        const int* off = p.state_only ? p.seg_off_nl : p.seg_off;
+        const int sgi = blockIdx.x / p.H, h = blockIdx.x % p.H;
+        if (sgi >= off[p.n_seq]) return;  // past the total: the whole CTA leaves before any barrier
+        int lo = 0, hi = p.n_seq;         // rank r with off[r] <= sgi < off[r + 1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (off[mid] <= sgi) lo = mid;
+            else hi = mid;
+        }
+        const int seq = p.order[lo];
+        const int t0 = p.cu_seqlens[seq] + (sgi - off[lo]) * p.seg_len;
+        len = max(0, min(p.seg_len, p.cu_seqlens[seq + 1] - t0));
+        row0 = (long)t0 * p.H + h;
+        row_stride = p.H;
+        if (p.state_only) {
+            state = (long)sgi * p.H + h;  // index of this segment's sum
+        } else {
+            state = (long)seq * p.H + h;
+            init = p.seg_init + ((long)sgi * p.H + h) * D * D;
+            init_t = false;
+            write_state = sgi == off[lo + 1] - 1;  // the sequence's last segment
+        }
     } else {
         const int seq = blockIdx.x / p.H, h = blockIdx.x % p.H;
         const int t0 = p.cu_seqlens[seq];

@@ -183,3 +183,44 @@ def test_ffma_workspace_size_follows_the_plan(la):
     assert la.prefill_workspace_size(1, 128, 65536, 128, torch.float32) == 0
     n = la.prefill_workspace_size(1, 8, 65536, 128, torch.float32)
     assert n > 0 and n % (8 * 128 * 128 * 4) == 0
+
+
+def _varlen_case(lens, H, d, seed, dtype="fp32", n_pool=2):
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    T = int(cu[-1])
+    q, k, v = synth.qkv((T, H, d), d, dtype, seed=seed)
+    pool = synth.outer_product_state(n_pool * H, d, d, [300] * (n_pool * H), seed=seed + 1).view(n_pool, H, d, d)
+    init = torch.tensor([(i % (n_pool + 1)) - 1 for i in range(len(lens))], dtype=torch.int32)
+    return cu, q, k, v, pool, init
+
+
+@pytest.mark.parametrize("lens,H,d", [([9000, 1, 0, 3000], 2, 128), ([20000], 1, 64), ([5000, 7000], 3, 128)])
+def test_ffma_varlen_auto_segments_match_oracle(la, oracle_mod, lens, H, d):
+    """A packed fp32 batch of few long sequences: one CTA per (segment, head)."""
+    cu, q, k, v, pool, init = _varlen_case(lens, H, d, seed=sum(lens) % 97 + d)
+    T = int(cu[-1])
+    base = la.prefill_varlen_workspace_size(len(lens), T, H, d, torch.float32)
+    assert base >= H * d * d * 4, "shape should be split (the workspace holds segment states)"
+    o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), pool.cuda(), init.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, init)
+    assert_out(o.cpu(), ro, torch.float32, 2)
+    assert_state(s.cpu(), rs, 1)
+
+
+@pytest.mark.parametrize("segments", ["2", "5"])
+def test_ffma_varlen_forced_segments_integer_bit_exact(la, oracle_mod, monkeypatch, segments):
+    monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    lens, H, d = [1500, 0, 700, 1], 2, 128
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    T = int(cu[-1])
+    q, k, v = (synth.integer_valued((T, H, d), seed=s) for s in (81, 82, 83))
+    pool = synth.integer_valued((2, H, d, d), seed=84, lo=-20, hi=20)
+    init = torch.tensor([1, 0, -1, 1], dtype=torch.int32)
+    o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), pool.cuda(), init.cuda())
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, init)
+    np.testing.assert_array_equal(to64(o.cpu()), ro)
+    np.testing.assert_array_equal(to64(s.cpu()), rs)
