@@ -577,24 +577,38 @@ def run_backward(args, dist: Dist, pk):
     return res
 
 
-def run_few_heads(args, dist: Dist, pk):
+# FFMA path: fused multiply-adds per token and head at d = 128, C = 64 (scores
+# on the diagonal half, outputs, state update: 0.28 M + 1.33 M + 1.05 M per
+# 64-token chunk), and the FP32 FFMA peak (148 SMs x 128 lanes x 2 FLOP x
+# 1.965 GHz)
+FFMA_FMA_PER_TOKEN_HEAD = (0.28e6 + 1.33e6 + 1.05e6) / 64
+FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_few_heads(args, dist: Dist, pk, dtype: str = "bf16"):
     """Long prefill with too few (batch, head) units to fill the GPU, once with
-    the library's segment split and once with it turned off."""
+    the library's segment split and once with it turned off (bf16 on the
+    tensor cores; fp32 on the FFMA path, over half the tokens)."""
     import long_context_linear_b200 as la
     import synth
     c = FEWHEADS
     B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    fp32 = dtype == "fp32"
+    if fp32:
+        N //= 2
+    tdt = torch.float32 if fp32 else torch.bfloat16
     dev = torch.device("cuda", torch.cuda.current_device())
-    q, k, v = synth.dense(B, H, N, d, "bf16", seed=71 + dist.rank, device=dev)
+    q, k, v = synth.dense(B, H, N, d, dtype, seed=71 + dist.rank, device=dev)
     o = torch.empty_like(v)
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    ws_bytes = la.prefill_workspace_size(B, H, N, d, torch.bfloat16)
+    ws_bytes = la.prefill_workspace_size(B, H, N, d, tdt)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     n = max(10, min(args.steps, 50))
-    res = dict(workload="prefill B=1 H=8 N=131072 d=128 bf16 (16 value-slice items on 148 SMs)",
+    items = "8 unit items" if fp32 else "16 value-slice items"
+    res = dict(workload=f"prefill B={B} H={H} N={N} d={d} {dtype} ({items} on 148 SMs)",
                workspace_bytes=ws_bytes, steps=n)
-    byts = prefill_bytes(B, H, N, d)
+    byts = prefill_bytes(B, H, N, d) + (4.0 * B * H * N * d * 2 if fp32 else 0)  # fp32 Q, K, V, O: twice the bytes
     prev = os.environ.get("LA_PREFILL_SEGMENTS")
     try:
         for key, env in (("split", None), ("unsplit", "1")):
@@ -608,6 +622,9 @@ def run_few_heads(args, dist: Dist, pk):
             gbs = byts / (ms_step / 1e3) / 1e9
             res[key] = dict(ms_per_step=ms_step, tokens_per_s=B * N * dist.world / (ms_step / 1e3), hbm_gbs=gbs,
                             frac=gbs / pk["hbm"])
+            if fp32:
+                tf = 2 * FFMA_FMA_PER_TOKEN_HEAD * B * H * N / (ms_step / 1e3) / 1e12
+                res[key].update(ffma_tflops=tf, ffma_frac=tf / FFMA_PEAK_TFLOPS)
     finally:
         if prev is None:
             os.environ.pop("LA_PREFILL_SEGMENTS", None)
@@ -728,6 +745,7 @@ def main():
         extras["prefill_8k_relu"] = run_prefill8k(args, dist, pk, "relu")
         extras["prefill_8k_d64"] = run_prefill8k(args, dist, pk, d=64)
         extras["few_heads"] = run_few_heads(args, dist, pk)
+        extras["few_heads_fp32"] = run_few_heads(args, dist, pk, "fp32")
         extras["backward_8k"] = run_backward(args, dist, pk)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
