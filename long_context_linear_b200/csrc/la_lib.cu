@@ -528,44 +528,41 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
 namespace {
 size_t varlen_order_bytes(int n_seq) { return n_seq > 0 ? round256((size_t)n_seq * sizeof(int)) : 0; }
 
-// Segment length (a multiple of C) for a packed batch whose (sequence, head,
-// value slice) items fill less than half of the SMs (`slices` per sequence and
-// head: d / 64 on the tensor cores, 1 on the FFMA path), or 0 for no split.  The host
-// knows only the total token count T, so segments are sized for T spread over
-// about one item per SM.  LA_PREFILL_SEGMENTS = P forces about P segments per
-// sequence of average length (1: no split).
-int plan_varlen_segments(int n_seq, int T, int H, int slices, int sms) {
+// Segment plan of a packed batch whose (sequence, head, value slice) items
+// fill less than half of the SMs (`slices` per sequence and head: d / 64 on
+// the tensor cores, 1 on the FFMA path): the most segments the batch may be
+// cut into (about one item per SM), or 0 for no split, and the shortest
+// segment (*min_seg tokens).  The host knows only the total token count T;
+// the device picks the segment length from the real lengths
+// (vorder::seg_plan_kernel).  With segments of at least min_seg tokens the
+// batch never has more than T / min_seg + n_seq of them, which bounds the
+// plan too.  LA_PREFILL_SEGMENTS = P allows P segments per sequence on
+// average, of at least one chunk (1: no split).
+long plan_varlen_segments(int n_seq, int T, int H, int slices, int sms, int* min_seg) {
+    *min_seg = kMinSegChunks * tc::C;
     if (n_seq <= 0 || T <= 0 || H <= 0) return 0;
-    const long C = tc::C;
+    long S;
     if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
-        const int P = atoi(e);
+        const long P = atol(e);
         if (P <= 1) return 0;
-        const long avg = ((long)T + n_seq - 1) / n_seq;
-        return (int)std::max(C, ((avg + P - 1) / P + C - 1) / C * C);
+        *min_seg = tc::C;
+        S = P * n_seq;
+    } else {
+        const long per_seq_items = (long)H * slices;
+        if ((long)n_seq * per_seq_items * 2 > sms) return 0;
+        S = sms / per_seq_items;  // segments that keep every item in one wave
+        if ((long)T < 2L * *min_seg) return 0;
     }
-    const long per_seq_items = (long)H * slices;
-    if ((long)n_seq * per_seq_items * 2 > sms) return 0;
-    // at most S segments keep every item in one wave; rounding each sequence
-    // up to whole segments adds at most one per sequence, so size for S - n_seq
-    const long S = sms / per_seq_items;
-    if (S <= 2L * n_seq) return 0;
-    const long target = S - n_seq;
-    const long seg = std::max((long)kMinSegChunks * C, (((long)T + target - 1) / target + C - 1) / C * C);
-    return (long)T >= 2 * seg ? (int)seg : 0;
+    S = std::min(S, (long)T / *min_seg + n_seq);
+    return S > n_seq ? S : 0;
 }
 
-// Upper bounds of the segment counts (all segments / all but each sequence's
-// last) and the bytes of the segment area: the two offset arrays, the
-// segment sums and the segment starts.
-void varlen_segment_counts(int n_seq, int T, int seg_len, long* max_segs, long* max_nl) {
-    *max_nl = T / seg_len;
-    *max_segs = *max_nl + n_seq;
-}
-size_t varlen_segment_bytes(int n_seq, int T, int H, int d, int seg_len) {
-    long ms, mnl;
-    varlen_segment_counts(n_seq, T, seg_len, &ms, &mnl);
+// Bytes of the segment area for at most max_segs segments: the two offset
+// arrays, the chosen segment length, the sums of all segments but each
+// sequence's last (at most max_segs - n_seq) and the segment starts.
+size_t varlen_segment_bytes(int n_seq, long max_segs, int H, int d) {
     const size_t state = (size_t)H * d * d * sizeof(float);
-    return 2 * round256((size_t)(n_seq + 1) * sizeof(int)) + (size_t)mnl * state + (size_t)ms * state;
+    return 2 * round256((size_t)(n_seq + 1) * sizeof(int)) + 256 + (size_t)(2 * max_segs - n_seq) * state;
 }
 }  // namespace
 
@@ -580,8 +577,9 @@ size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int 
     size_t total = base + (tc ? phi_workspace_bytes((long)T * H, dk, phi) : 0);
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return total;
-    const int seg_len = plan_varlen_segments(n_seq, T, H, tc ? tc_slices(dk) : 1, di->sms);
-    if (seg_len) total += varlen_segment_bytes(n_seq, T, H, dk, seg_len);
+    int min_seg;
+    const long max_segs = plan_varlen_segments(n_seq, T, H, tc ? tc_slices(dk) : 1, di->sms, &min_seg);
+    if (max_segs) total += varlen_segment_bytes(n_seq, max_segs, H, dk);
     return total;
 }
 
@@ -650,11 +648,10 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         };
         // the segment split as on the tensor cores (one item per sequence and
         // head), when the workspace has room for the order and the segment area
-        const int seg_len = plan_varlen_segments(n_seq, T, H, 1, di->sms);
-        long max_segs = 0, max_nl = 0;
-        if (seg_len) varlen_segment_counts(n_seq, T, seg_len, &max_segs, &max_nl);
-        if (!seg_len || !workspace || !aligned16(workspace) || max_segs * H > (1L << 30) ||
-            ws_bytes < need + varlen_segment_bytes(n_seq, T, H, dk, seg_len))
+        int min_seg;
+        const long max_segs = plan_varlen_segments(n_seq, T, H, 1, di->sms, &min_seg), max_nl = max_segs - n_seq;
+        if (!max_segs || !workspace || !aligned16(workspace) || max_segs * H > (1L << 30) ||
+            ws_bytes < need + varlen_segment_bytes(n_seq, max_segs, H, dk))
             return go(sp, (long)n_seq * H);
         int* order = reinterpret_cast<int*>(workspace);
         vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
@@ -663,15 +660,17 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         const size_t ints = round256((size_t)(n_seq + 1) * sizeof(int));
         int* seg_off = reinterpret_cast<int*>(w);
         int* seg_off_nl = reinterpret_cast<int*>(w + ints);
-        float* sums = reinterpret_cast<float*>(w + 2 * ints);
+        int* seg_len = reinterpret_cast<int*>(w + 2 * ints);
+        float* sums = reinterpret_cast<float*>(w + 2 * ints + 256);
         float* starts = sums + (size_t)max_nl * H * dk * dv;
-        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, seg_len, seg_off, seg_off_nl);
+        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, max_segs, min_seg, tc::C, seg_len, seg_off,
+                                                  seg_off_nl);
         if ((s = after_launch("varlen segment plan launch")) != LA_OK) return s;
         sp.order = order;
         sp.seg_off = seg_off;
         sp.seg_off_nl = seg_off_nl;
         sp.n_seq = n_seq;
-        sp.seg_len = seg_len;
+        sp.seg_len_dev = seg_len;
         if (max_nl > 0) {
             simt::Params p1 = sp;
             p1.state_only = 1;
@@ -702,12 +701,12 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         off_seg += ws_phi;
     }
     const int nvs = tc_slices(dv);
-    int seg_len = plan_varlen_segments(n_seq, T, H, nvs, di->sms);
-    long max_segs = 0, max_nl = 0;
-    if (seg_len) varlen_segment_counts(n_seq, T, seg_len, &max_segs, &max_nl);
-    if (seg_len && (ws_bytes < off_seg + varlen_segment_bytes(n_seq, T, H, dk, seg_len) ||
-                    max_segs * H * nvs > (1L << 30)))
-        seg_len = 0;  // no room for the segment states: whole sequences
+    int min_seg;
+    long max_segs = plan_varlen_segments(n_seq, T, H, nvs, di->sms, &min_seg);
+    if (max_segs && (ws_bytes < off_seg + varlen_segment_bytes(n_seq, max_segs, H, dk) ||
+                     max_segs * H * nvs > (1L << 30)))
+        max_segs = 0;  // no room for the segment states: whole sequences
+    const long max_nl = max_segs - n_seq;
 
     tc::Params p{};
     p.mode = 1;
@@ -732,21 +731,24 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     if ((s = make_map(&mk, k ? k : any, dk, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
     if ((s = make_map(&mv, v ? v : any, dv, H, Tm, head, tok, 1, tc::C)) != LA_OK) return s;
     if ((s = make_map(&mo, o ? o : any, dv, H, Tm, head, tok, 1, 32)) != LA_OK) return s;
-    if (seg_len) {
-        // segments: offsets in work order, the sums of all but each sequence's
-        // last segment, the state before every segment, then every segment
+    if (max_segs) {
+        // segments: the plan (length, offsets in work order), the sums of all
+        // but each sequence's last segment, the state before every segment,
+        // then every segment
         uint8_t* w = reinterpret_cast<uint8_t*>(workspace) + off_seg;
         const size_t ints = round256((size_t)(n_seq + 1) * sizeof(int));
         int* seg_off = reinterpret_cast<int*>(w);
         int* seg_off_nl = reinterpret_cast<int*>(w + ints);
-        float* sums = reinterpret_cast<float*>(w + 2 * ints);
+        int* seg_len = reinterpret_cast<int*>(w + 2 * ints);
+        float* sums = reinterpret_cast<float*>(w + 2 * ints + 256);
         float* starts = sums + (size_t)max_nl * H * dk * dv;
-        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, seg_len, seg_off, seg_off_nl);
+        vorder::seg_plan_kernel<<<1, 32, 0, st>>>(cu_seqlens, order, n_seq, max_segs, min_seg, tc::C, seg_len, seg_off,
+                                                  seg_off_nl);
         if ((s = after_launch("varlen segment plan launch")) != LA_OK) return s;
         p.seg_off = seg_off;
         p.seg_off_nl = seg_off_nl;
         p.n_seq = n_seq;
-        p.seg_len = seg_len;
+        p.seg_len_dev = seg_len;
         if (max_nl > 0) {
             tc::Params p1 = p;
             p1.state_only = 1;

@@ -49,14 +49,15 @@ struct Params {
     const float* seg_init;  // [U][n_seg][d][d]: state before each segment, or null
     int s_out_per_seg;      // 1: s_out is [U][n_seg][d][d], one state per segment
     int state_only;         // 1: only S = (init) + sum K^T V over the segment
-    // packed only: segments of seg_len tokens, CTA = segment * H + head, with
-    // the segments numbered in the work order of `order` (vorder::
-    // seg_plan_kernel offsets over n_seq sequences); a state-only launch numbers
+    // packed only: segments of *seg_len_dev tokens, CTA = segment * H + head,
+    // with the segments numbered in the work order of `order` (the length and
+    // the offsets over n_seq sequences from vorder::seg_plan_kernel); a state-only launch numbers
     // only the segments that are not a sequence's last (seg_off_nl).  CTAs past
     // the device-side total (the host launches an upper bound) do nothing.
     const int* order;
     const int* seg_off;
     const int* seg_off_nl;
+    const int* seg_len_dev;
     int n_seq;
 };
 
@@ -220,9 +221,9 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             if (off[mid] <= sgi) lo = mid;
             else hi = mid;
         }
-        const int seq = p.order[lo];
-        const int t0 = p.cu_seqlens[seq] + (sgi - off[lo]) * p.seg_len;
-        len = max(0, min(p.seg_len, p.cu_seqlens[seq + 1] - t0));
+        const int seq = p.order[lo], sl = *p.seg_len_dev;
+        const int t0 = p.cu_seqlens[seq] + (sgi - off[lo]) * sl;
+        len = max(0, min(sl, p.cu_seqlens[seq + 1] - t0));
         row0 = (long)t0 * p.H + h;
         row_stride = p.H;
         if (p.state_only) {

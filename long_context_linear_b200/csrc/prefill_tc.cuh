@@ -119,10 +119,11 @@ struct Params {
     int init_transposed;   // the initial state is given as its transpose [dv][DK]
     int seg_base;          // dense: the items' segments are seg_base .. seg_base + n_seg - 1
     int dk;                // key dim = value dim: 128 or 64 (selects the kernel instance)
-    // packed only: segments of seg_len tokens (vorder::seg_plan_kernel offsets
-    // in work order over n_seq sequences), or null
+    // packed only: segments of *seg_len_dev tokens (the length and the offsets
+    // in work order over n_seq sequences from vorder::seg_plan_kernel), or null
     const int* seg_off;
     const int* seg_off_nl;
+    const int* seg_len_dev;
     int n_seq;
 };
 
@@ -199,9 +200,9 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
             }
             const int r = lo, sg = sgi - off[r];
             const int seq = p.order[r];
-            const int end = p.cu_seqlens[seq + 1];
-            it.t0 = p.cu_seqlens[seq] + sg * p.seg_len;
-            it.len = max(0, min(p.seg_len, end - it.t0));
+            const int end = p.cu_seqlens[seq + 1], sl = *p.seg_len_dev;
+            it.t0 = p.cu_seqlens[seq] + sg * sl;
+            it.len = max(0, min(sl, end - it.t0));
             if (p.state_only) {
                 it.state = (long)sgi * p.H + h;  // index of this segment's sum
                 it.init = nullptr;

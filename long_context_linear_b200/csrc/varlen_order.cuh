@@ -29,16 +29,45 @@ __global__ void __launch_bounds__(NUM_THREADS) order_kernel(const int* __restric
     }
 }
 
-// Segments of a packed batch cut into pieces of seg_len tokens (the last piece
-// of a sequence may be shorter; an empty sequence keeps one empty piece).  In
-// work order (rank r = position in `order`): seg_off[r] = the number of
-// segments before rank r, seg_off_nl[r] = the same not counting each
-// sequence's last segment; both have n_seq + 1 entries.  One warp scans the
-// ranks 32 at a time.
+// Segments of a packed batch: the segment length is chosen here, where the
+// lengths are known, as the smallest multiple of `unit` tokens, at least
+// min_seg, for which the batch has at most max_segs segments (a sequence of
+// len tokens has max(1, ceil(len / seg_len)) of them; the last one may be
+// shorter; an empty sequence keeps one empty piece).  max_segs >= n_seq.
+// Written: *seg_len, and in work order (rank r = position in `order`):
+// seg_off[r] = the number of segments before rank r, seg_off_nl[r] = the same
+// not counting each sequence's last segment; both have n_seq + 1 entries.
+// One warp: a binary search over the length, then a scan of the ranks 32 at a
+// time.
+__device__ __forceinline__ int seg_pieces(int len, int seg) {
+    return static_cast<int>(max(1L, ((long)len + seg - 1) / seg));
+}
+__device__ __forceinline__ long seg_count_warp(const int* __restrict__ cu, int n_seq, int seg) {
+    long c = 0;
+    for (int i = threadIdx.x; i < n_seq; i += 32) c += seg_pieces(cu[i + 1] - cu[i], seg);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    return c;
+}
+
 __global__ void __launch_bounds__(32) seg_plan_kernel(const int* __restrict__ cu, const int* __restrict__ order,
-                                                     int n_seq, int seg_len, int* __restrict__ seg_off,
+                                                     int n_seq, long max_segs, int min_seg, int unit,
+                                                     int* __restrict__ seg_len_out, int* __restrict__ seg_off,
                                                      int* __restrict__ seg_off_nl) {
     const int lane = threadIdx.x;
+    int max_len = 0;
+    for (int i = lane; i < n_seq; i += 32) max_len = max(max_len, cu[i + 1] - cu[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) max_len = max(max_len, __shfl_xor_sync(0xffffffffu, max_len, off));
+    // smallest u in [lo, hi] with count(u * unit) <= max_segs; count(hi * unit) = n_seq
+    int lo = (min_seg + unit - 1) / unit, hi = max(lo, (max_len + unit - 1) / unit);
+    while (lo < hi) {
+        const int mid = lo + (hi - lo) / 2;
+        if (seg_count_warp(cu, n_seq, mid * unit) <= max_segs) hi = mid;
+        else lo = mid + 1;
+    }
+    const int seg_len = lo * unit;
+    if (lane == 0) *seg_len_out = seg_len;
     int carry = 0, carry_nl = 0;
     for (int base = 0; base < n_seq; base += 32) {
         const int r = base + lane;
@@ -46,7 +75,7 @@ __global__ void __launch_bounds__(32) seg_plan_kernel(const int* __restrict__ cu
         if (r < n_seq) {
             const int sq = order[r];
             const int len = cu[sq + 1] - cu[sq];
-            c = max(1, (len + seg_len - 1) / seg_len);
+            c = seg_pieces(len, seg_len);
         }
         const int cnl = r < n_seq ? c - 1 : 0;
         int x = c, y = cnl;  // inclusive scans over the warp
