@@ -17,8 +17,9 @@
 //
 // A feature map phi (phi.cuh) is applied to q and k as they are loaded.
 // Both read the d x d fp32 state once (commit also writes it): 3 state passes
-// for m tokens instead of 2 m with m decode steps.  Layout per unit as in
-// decode.cuh: thread = one 16-byte column vector of D/RS rows.
+// for m tokens instead of 2 m with m decode steps.  Commit keeps the layout of
+// decode.cuh (thread = one 16-byte column vector of D/RS rows); verify streams
+// the rows (below).
 #pragma once
 #include <cuda_bf16.h>
 #include "decode.cuh"
@@ -28,8 +29,6 @@ namespace dmulti {
 
 constexpr int NUM_THREADS = 256;
 constexpr int MAX_M = 16;
-
-constexpr int G = 4;  // draft tokens per reduction round of verify
 
 // 16 bytes of T -> fp32 (4 fp32 or 8 bf16 values)
 __device__ __forceinline__ void unpack16(const uint4 r, float (&f)[4]) {
@@ -44,51 +43,77 @@ __device__ __forceinline__ void unpack16(const uint4 r, float (&f)[8]) {
     }
 }
 
-// Two CTAs per SM: the bound lets the compiler use up to 128 registers, and
-// with them verify keeps more loads in flight (measured: 0.213 ms against
-// 0.257 ms at 101 registers for B=256, H=64, m=4).
-template <typename T, int D>
-__global__ void __launch_bounds__(NUM_THREADS, 2)
+// 4 values at dst: 16 bytes of fp32 or 8 bytes of bf16 (nearest even)
+__device__ __forceinline__ void store4(float* dst, const float4 y) { *reinterpret_cast<float4*>(dst) = y; }
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, const float4 y) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(y.x, y.y), b = __floats2bfloat162_rn(y.z, y.w);
+    *reinterpret_cast<uint2*>(dst) = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
+
+// verify, one CTA of D / 2 threads per unit, in two row groups of D / 4:
+// thread (g, c) owns value columns 4c .. 4c + 3 and rows g * D / 2 .. of S_0,
+// which it streams from HBM one 16-byte piece per row (8 rows in flight),
+// updating the q_t S_0 sums of all MB drafts per piece.  q is also stored
+// transposed, draft index fastest, so that four drafts' q_i come in one
+// broadcast load.  Row group 1 hands its partial sums to group 0 through
+// shared memory; group 0 adds them and the intra-draft terms and stores o.
+// MB = 4, 8 or 16 >= m (drafts past m are zero and not stored).  Keeping a
+// second batch of rows in flight per thread was measured slower (its
+// registers cost more occupancy than the overlap gained: m = 16, 0.739 ms
+// against 0.664).
+template <typename T, int D, int MB>
+__global__ void __launch_bounds__(D / 2)
 verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
               const float* __restrict__ S, int m, int phi) {
-    constexpr int TPR = D / 4;
-    constexpr int RS = NUM_THREADS / TPR;
-    constexpr int RPT = D / RS;
-    __shared__ __align__(16) float qs[MAX_M][D], ks[MAX_M][D], vs[MAX_M][D];
-    __shared__ float A[MAX_M][MAX_M];  // A[t][s] = q_t . k_s, s <= t
-    __shared__ __align__(16) float red[G][RS][D];
+    constexpr int LPR = D / 4;  // threads per row group
+    constexpr int NT = 2 * LPR;
+    constexpr int ROWS = D / 2;  // rows per group
+    constexpr int UNR = 8;       // rows in flight per thread
+    static_assert(ROWS % UNR == 0 && MB % 4 == 0 && MB <= MAX_M, "verify layout");
+    __shared__ __align__(16) float qT[D][MB];
+    __shared__ __align__(16) float qs[MB][D], ks[MB][D], vs[MB][D];
+    __shared__ float A[MB][MB];  // A[t][s] = q_t . k_s, s <= t
+    __shared__ __align__(16) float red[MB][D];
 
     const long u = blockIdx.x;
-    const int tid = threadIdx.x;
-    const int c4 = tid % TPR, slot = tid / TPR;
-    const float4* Su = reinterpret_cast<const float4*>(S + u * D * D);
-    float4 x[RPT];
+    const int tid = threadIdx.x, g = tid / LPR, c = tid % LPR;
+    // the first rows of S_0 are requested before the drafts are read
+    const float4* Sg = reinterpret_cast<const float4*>(S + u * D * D) + (long)g * ROWS * LPR + c;
+    float4 x[UNR];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) x[r] = __ldcs(&Su[(slot + r * RS) * TPR + c4]);
+    for (int j = 0; j < UNR; ++j) x[j] = __ldcs(Sg + (long)j * LPR);
+    // the drafts' q, k, v (phi on q and k), zero past m; 16-byte loads
     const long base = u * (long)m * D;
-    // the drafts' q, k, v: 16-byte loads (rows are 16-byte aligned: D * sizeof(T) is)
     constexpr int VEC = 16 / (int)sizeof(T);
-    for (int e = tid * VEC; e < m * D; e += NUM_THREADS * VEC) {
+    for (int e = tid * VEC; e < MB * D; e += NT * VEC) {
         const int t = e / D, i = e % D;
         float qv[VEC], kv[VEC], vv[VEC];
-        unpack16(*reinterpret_cast<const uint4*>(q + base + e), qv);
-        unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
-        unpack16(*reinterpret_cast<const uint4*>(v + base + e), vv);
+        if (t < m) {
+            unpack16(*reinterpret_cast<const uint4*>(q + base + e), qv);
+            unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
+            unpack16(*reinterpret_cast<const uint4*>(v + base + e), vv);
 #pragma unroll
-        for (int j = 0; j < VEC; j += 4) {
-            *reinterpret_cast<float4*>(&qs[t][i + j]) = make_float4(apply_phi(qv[j], phi), apply_phi(qv[j + 1], phi),
-                                                                    apply_phi(qv[j + 2], phi), apply_phi(qv[j + 3], phi));
-            *reinterpret_cast<float4*>(&ks[t][i + j]) = make_float4(apply_phi(kv[j], phi), apply_phi(kv[j + 1], phi),
-                                                                    apply_phi(kv[j + 2], phi), apply_phi(kv[j + 3], phi));
-            *reinterpret_cast<float4*>(&vs[t][i + j]) = make_float4(vv[j], vv[j + 1], vv[j + 2], vv[j + 3]);
+            for (int jj = 0; jj < VEC; ++jj) {
+                qv[jj] = apply_phi(qv[jj], phi);
+                kv[jj] = apply_phi(kv[jj], phi);
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < VEC; ++jj) qv[jj] = kv[jj] = vv[jj] = 0.f;
         }
+#pragma unroll
+        for (int jj = 0; jj < VEC; jj += 4) {
+            *reinterpret_cast<float4*>(&qs[t][i + jj]) = make_float4(qv[jj], qv[jj + 1], qv[jj + 2], qv[jj + 3]);
+            *reinterpret_cast<float4*>(&ks[t][i + jj]) = make_float4(kv[jj], kv[jj + 1], kv[jj + 2], kv[jj + 3]);
+            *reinterpret_cast<float4*>(&vs[t][i + jj]) = make_float4(vv[jj], vv[jj + 1], vv[jj + 2], vv[jj + 3]);
+        }
+#pragma unroll
+        for (int jj = 0; jj < VEC; ++jj) qT[i + jj][t] = qv[jj];
     }
     __syncthreads();
-    // intra-draft scores: one warp per pair (t, s), s <= t, lanes split the dim;
-    // pairs in row order, warp w taking every 8th from the w-th, (t, s) stepped
-    // along without recomputing it from the pair index
+    // intra-draft scores: one warp per pair (t, s), s <= t, lanes split the dim
     {
-        constexpr int NW = NUM_THREADS / 32;
+        constexpr int NW = NT / 32 > 0 ? NT / 32 : 1;
         const int warp = tid >> 5, lane = tid & 31;
         int t = 0, s = warp;
         while (s > t) { s -= t + 1; ++t; }
@@ -103,36 +128,56 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
             while (s > t) { s -= t + 1; ++t; }
         }
     }
-    // q_t S_0 for G draft tokens at a time, reduced over row slots, plus the
-    // intra-draft terms (A is complete after the barrier below)
-    for (int t0 = 0; t0 < m; t0 += G) {
-        const int gn = min(G, m - t0);
-        float4 acc[G];
+    // q_t S_0 over this group's rows for all MB drafts
+    float4 acc[MB];
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < MB; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int r0 = 0; r0 < ROWS; r0 += UNR) {
+        if (r0 > 0) {
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) {
+            for (int j = 0; j < UNR; ++j) x[j] = __ldcs(Sg + (long)(r0 + j) * LPR);
+        }
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float qi = g < gn ? qs[t0 + g][slot + r * RS] : 0.f;
-                acc[g].x = fmaf(qi, x[r].x, acc[g].x);
-                acc[g].y = fmaf(qi, x[r].y, acc[g].y);
-                acc[g].z = fmaf(qi, x[r].z, acc[g].z);
-                acc[g].w = fmaf(qi, x[r].w, acc[g].w);
+        for (int j = 0; j < UNR; ++j) {
+            const float* qrow = qT[g * ROWS + r0 + j];
+#pragma unroll
+            for (int t4 = 0; t4 < MB; t4 += 4) {
+                const float4 qq = *reinterpret_cast<const float4*>(qrow + t4);
+                const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    float4& a = acc[t4 + tt];
+                    a.x = fmaf(qa[tt], x[j].x, a.x);
+                    a.y = fmaf(qa[tt], x[j].y, a.y);
+                    a.z = fmaf(qa[tt], x[j].z, a.z);
+                    a.w = fmaf(qa[tt], x[j].w, a.w);
+                }
             }
         }
+    }
+    if (g == 1) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) *reinterpret_cast<float4*>(&red[g][slot][4 * c4]) = acc[g];
-        __syncthreads();
-        for (int e = tid; e < gn * D; e += NUM_THREADS) {
-            const int g = e / D, col = e % D, t = t0 + g;
-            float sum = 0.f;
+        for (int t = 0; t < MB; ++t) *reinterpret_cast<float4*>(&red[t][4 * c]) = acc[t];
+    }
+    __syncthreads();
+    if (g == 0) {
 #pragma unroll
-            for (int sl = 0; sl < RS; ++sl) sum += red[g][sl][col];
-            for (int s = 0; s <= t; ++s) sum = fmaf(A[t][s], vs[s][col], sum);
-            dec::st_f(o + base + (long)t * D + col, sum);
+        for (int t = 0; t < MB; ++t) {
+            if (t < m) {
+                const float4 p = *reinterpret_cast<const float4*>(&red[t][4 * c]);
+                float4 y = make_float4(acc[t].x + p.x, acc[t].y + p.y, acc[t].z + p.z, acc[t].w + p.w);
+                for (int s = 0; s <= t; ++s) {
+                    const float a = A[t][s];
+                    const float4 vv = *reinterpret_cast<const float4*>(&vs[s][4 * c]);
+                    y.x = fmaf(a, vv.x, y.x);
+                    y.y = fmaf(a, vv.y, y.y);
+                    y.z = fmaf(a, vv.z, y.z);
+                    y.w = fmaf(a, vv.w, y.w);
+                }
+                store4(o + base + (long)t * D + 4 * c, y);
+            }
         }
-        __syncthreads();
     }
 }
 

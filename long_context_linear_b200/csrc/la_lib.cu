@@ -256,6 +256,21 @@ void launch_decode(int dk, int grid, const void* q, const void* k, const void* v
 
 namespace lcl {
 namespace {
+// verify for m drafts: the instance for the smallest draft capacity MB >= m
+template <typename T, int D>
+void launch_verify_d(int m, int grid, const T* q, const T* k, const T* v, T* o, const float* S, int phi,
+                     cudaStream_t st) {
+    if (m <= 4) dmulti::verify_kernel<T, D, 4><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else if (m <= 8) dmulti::verify_kernel<T, D, 8><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else dmulti::verify_kernel<T, D, 16><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+}
+template <typename T>
+void launch_verify(int dk, int m, int grid, const void* q, const void* k, const void* v, void* o, const float* S,
+                   int phi, cudaStream_t st) {
+    if (dk == 128) launch_verify_d<T, 128>(m, grid, (const T*)q, (const T*)k, (const T*)v, (T*)o, S, phi, st);
+    else launch_verify_d<T, 64>(m, grid, (const T*)q, (const T*)k, (const T*)v, (T*)o, S, phi, st);
+}
+
 template <typename T, int D>
 void launch_commit_d(int m, int grid, const T* k, const T* v, float* S, const int32_t* accepted, int H, int phi,
                      cudaStream_t st) {
@@ -832,16 +847,8 @@ la_status la_decode_verify(const void* q, const void* k, const void* v, void* o,
     DeviceInfo* di;
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int grid = (int)U;
-    if (dt == LA_BF16) {
-        using T = __nv_bfloat16;
-        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
-        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
-    } else {
-        using T = float;
-        if (dk == 128) dmulti::verify_kernel<T, 128><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
-        else dmulti::verify_kernel<T, 64><<<grid, dmulti::NUM_THREADS, 0, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, S, m, phi);
-    }
+    if (dt == LA_BF16) launch_verify<__nv_bfloat16>(dk, m, (int)U, q, k, v, o, S, phi, st);
+    else launch_verify<float>(dk, m, (int)U, q, k, v, o, S, phi, st);
     return after_launch("decode_verify launch");
 }
 
