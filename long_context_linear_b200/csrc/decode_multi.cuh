@@ -57,7 +57,7 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float4 y) {
 // transposed, draft index fastest, so that four drafts' q_i come in one
 // broadcast load.  Row group 1 hands its partial sums to group 0 through
 // shared memory; group 0 adds them and the intra-draft terms and stores o.
-// MB = 4, 8 or 16 >= m (drafts past m are zero and not stored).  Keeping a
+// MB = 4, 8, 12 or 16 >= m (drafts past m are zero and not stored).  Keeping a
 // second batch of rows in flight per thread was measured slower (its
 // registers cost more occupancy than the overlap gained: m = 16, 0.739 ms
 // against 0.664).

@@ -262,6 +262,7 @@ void launch_verify_d(int m, int grid, const T* q, const T* k, const T* v, T* o, 
                      cudaStream_t st) {
     if (m <= 4) dmulti::verify_kernel<T, D, 4><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
     else if (m <= 8) dmulti::verify_kernel<T, D, 8><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else if (m <= 12) dmulti::verify_kernel<T, D, 12><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
     else dmulti::verify_kernel<T, D, 16><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
 }
 template <typename T>

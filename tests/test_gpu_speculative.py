@@ -30,8 +30,8 @@ def _case(B, H, m, d, dtype, seed):
     return S, q, k, v
 
 
-@pytest.mark.parametrize("m", [1, 2, 4, 7, 16])
-@pytest.mark.parametrize("d,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp32")])
+@pytest.mark.parametrize("m", [1, 2, 4, 7, 8, 10, 12, 13, 16])  # every draft-capacity instance (4, 8, 12, 16)
+@pytest.mark.parametrize("d,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp32"), (64, "fp32")])
 def test_verify_matches_recurrence_over_drafts(la, oracle_mod, m, d, dtype):
     B, H = 3, 4
     S, q, k, v = _case(B, H, m, d, dtype, seed=m * 10 + d)
