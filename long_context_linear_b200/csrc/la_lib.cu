@@ -138,7 +138,7 @@ la_status encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
 // 3-D bf16 tensor map with a 64-element (128-byte) inner box and 128B swizzle.
 la_status make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
                    uint64_t stride2_bytes, uint32_t b1, uint32_t b2) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     la_status s = encoder(&enc);
     if (s != LA_OK) return s;
     cuuint64_t dims[3] = {d0, d1, d2};

@@ -1,6 +1,5 @@
 """The C-ABI library loads without a GPU, exports every symbol include/la.h
 declares, and rejects bad arguments on the host before touching the device."""
-import ctypes
 import os
 import re
 

@@ -4,12 +4,11 @@ Each test runs the whole batch through the C ABI exactly as the benchmark does
 (same shapes, same calls) and compares seeded samples of (batch, head) units
 against the fp64 oracle, which computes those units one by one.
 """
-import numpy as np
 import pytest
 import torch
 
 import synth
-from tests.parity import assert_out, assert_state, to64
+from tests.parity import assert_out, assert_state
 
 pytestmark = pytest.mark.gpu
 

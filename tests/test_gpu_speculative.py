@@ -7,7 +7,6 @@ verify's outputs against the fp64 recurrence run over the m drafts from S;
 commit's state against the recurrence over the accepted prefix, and bit for
 bit against the same number of la_decode_step calls.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -1,5 +1,4 @@
 """Packed ragged prefill with prefix resume on the GPU against the fp64 oracle."""
-import os
 
 import numpy as np
 import pytest
