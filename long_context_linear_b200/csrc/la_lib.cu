@@ -305,7 +305,7 @@ const char* la_status_string(la_status s) {
 
 const char* la_last_error(void) { return g_last_error; }
 
-int la_version(void) { return 200; }  // 0.2.0
+int la_version(void) { return 300; }  // 0.3.0
 
 namespace {
 
