@@ -73,7 +73,7 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     __shared__ __align__(16) float qT[D][MB];
     __shared__ __align__(16) float qs[MB][D], ks[MB][D], vs[MB][D];
     __shared__ float A[MB][MB];  // A[t][s] = q_t . k_s, s <= t
-    __shared__ __align__(16) float red[MB][D];
+    float(*red)[D] = qs;         // group 1's partial sums, once the scores are done with q
 
     const long u = blockIdx.x;
     const int tid = threadIdx.x, g = tid / LPR, c = tid % LPR;
@@ -128,6 +128,7 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
             while (s > t) { s -= t + 1; ++t; }
         }
     }
+    __syncthreads();  // qs is reused for the partial sums below
     // q_t S_0 over this group's rows for all MB drafts
     float4 acc[MB];
 #pragma unroll
