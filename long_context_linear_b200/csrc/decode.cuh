@@ -133,9 +133,14 @@ __host__ __device__ constexpr int decode_threads() { return Vec<SS>::E >= 8 ? NU
 // CTAs per SM the register budget is sized for.  8-bit states: 8 (64
 // registers, a 60-byte spill) against the 6 that their 80 registers allow
 // otherwise; measured 5-7 % faster on B=256, H=64 (e4m3 and e5m2, either
-// launch order), with bit-identical states.
+// launch order), with bit-identical states.  16-bit states: 5 (96 registers)
+// and fp32: 3 (80): a bound of 1 let the compiler take them to 168 and 96
+// registers, which measured 6 % slower (fp32 state 0.338 against 0.319 ms,
+// bf16 0.172 against 0.163 ms per step).
 template <typename SS>
-__host__ __device__ constexpr int decode_min_blocks() { return Vec<SS>::E == 16 ? 8 : 1; }
+__host__ __device__ constexpr int decode_min_blocks() {
+    return Vec<SS>::E == 16 ? 8 : (Vec<SS>::E == 8 ? 5 : 3);
+}
 
 template <typename T, typename SS, int D>
 __global__ void __launch_bounds__(decode_threads<SS>(), decode_min_blocks<SS>())
