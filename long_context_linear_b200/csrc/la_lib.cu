@@ -99,7 +99,7 @@ la_status device_info(DeviceInfo** out) {
         int major = 0;
         if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
             return cuda_fail(e, "cudaDeviceGetAttribute");
-        if (major != 10) return fail(LA_ERR_UNSUPPORTED, "device %d is sm_%d x, this build targets sm_100a", dev, major);
+        if (major != 10) return fail(LA_ERR_UNSUPPORTED, "device %d is sm_%d x; the library is compiled for sm_100a", dev, major);
         if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail(e, "cudaDeviceGetAttribute");
         if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word)) != cudaSuccess)
