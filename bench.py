@@ -7,10 +7,14 @@ One step = one la_prefill call over that batch; value = prefill tokens/s
 (B*N tokens per step, all ranks summed).  Inputs (6 GiB) are larger than L2,
 so no flush is needed between steps.
 
-Also reported in the same line (same timing rules): the batched decode step
-(B=256, H=64, d=128, 1024 consecutive steps, achieved HBM GB/s), the ragged
-varlen prefill with prefix resume (64 sequences, lengths ~U[1K,32K], H=32)
-and the B=4, H=32, N=8192 prefill.
+Also measured (same timing rules): the batched decode step (B=256, H=64,
+d=128, 1024 consecutive steps, achieved HBM GB/s), the ragged varlen prefill
+with prefix resume (64 sequences, lengths ~U[1K,32K], H=32), the B=4, H=32,
+N=8192 prefill, the fp32 B=1, H=2, N=256, d=64 configuration and further
+variants, each beside the fp64 oracle timed on the host cores on a bounded
+sample of the same workload.  Their detailed figures go on a line of their own
+({"bench_extras": ...}) before the headline line, and the headline line ends
+with a compact "summary" of them.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
 headline workload instead (rank 0 only).
@@ -287,7 +291,7 @@ def run_headline(args, dist: Dist, pk, sampler: ClockSampler):
     return res, sample
 
 
-def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
+def run_decode(args, dist: Dist, pk, state_dtype=torch.float32, cpu=False):
     import long_context_linear_b200 as la
     import synth
     c = DECODE
@@ -305,6 +309,11 @@ def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
     os_ = torch.empty_like(vs)
     stream = torch.cuda.current_stream(dev)
     it = [0]
+    sample = None
+    if cpu and state_dtype == torch.float32:
+        # the same starting states and tokens of a seeded sample of units, for the oracle
+        units = torch.tensor(synth.choose(U, CPU_DECODE_UNITS, seed=3), device=dev)
+        sample = (S.view(U, d, d)[units].cpu(),) + tuple(x.view(steps, U, d)[:, units].cpu() for x in (qs, ks, vs))
 
     def step():
         t = it[0] % steps
@@ -322,9 +331,12 @@ def run_decode(args, dist: Dist, pk, state_dtype=torch.float32):
     torch.cuda.empty_cache()
     name = {torch.float32: "fp32", torch.bfloat16: "bf16", torch.float16: "fp16",
             torch.float8_e4m3fn: "fp8_e4m3", torch.float8_e5m2: "fp8_e5m2"}[state_dtype]
-    return dict(workload=f"decode B=256 H=64 d=128 bf16 q/k/v, {name} state, 1024 consecutive steps",
-                hbm_gbs=gbs, peak_gbs=pk["hbm"], frac=gbs / pk["hbm"], ms_per_step=ms_step,
-                bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
+    res = dict(workload=f"decode B=256 H=64 d=128 bf16 q/k/v, {name} state, 1024 consecutive steps",
+               hbm_gbs=gbs, peak_gbs=pk["hbm"], frac=gbs / pk["hbm"], ms_per_step=ms_step,
+               bytes_per_step=bytes_step, tokens_per_s=B * dist.world / (ms_step / 1e3), steps=steps)
+    if sample is not None:
+        res["cpu_baseline"] = oracle_decode_baseline(*sample, H)
+    return res
 
 
 def run_decode_small_graph(args, dist: Dist, pk):
@@ -417,7 +429,7 @@ def run_speculative(args, dist: Dist, pk, m: int = 4):
                 rounds=rounds)
 
 
-def run_varlen(args, dist: Dist, pk):
+def run_varlen(args, dist: Dist, pk, cpu=False):
     import long_context_linear_b200 as la
     import synth
     c = VARLEN
@@ -448,14 +460,21 @@ def run_varlen(args, dist: Dist, pk):
     ms_step = total_ms / n
     byts = 4.0 * T * H * d * 2 + c["n_seq"] * H * d * d * 4 + c["n_resume"] * H * d * d * 4
     gbs = byts / (ms_step / 1e3) / 1e9
+    res = dict(workload="varlen 64 seqs len~U[1K,32K] (T=%d), H=32, d=128, bf16, 32 resumed from fp32 states" % T,
+               tokens_per_s=T * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
+               frac=gbs / pk["hbm"], tflops_rec=flops_rec(T * H, d) / (ms_step / 1e3) / 1e12, steps=n)
+    if cpu:
+        seqs = synth.choose(c["n_seq"], CPU_VARLEN_SEQS, seed=4)
+        cuh = cu.cpu()
+        parts = [(int(cuh[n]), int(cuh[n + 1]), int(idx[n])) for n in seqs]
+        sub = [tuple(x[a:b].cpu() for x in (q, k, v)) for a, b, _ in parts]
+        res["cpu_baseline"] = oracle_varlen_baseline(sub, [i for _, _, i in parts], pool.cpu())
     del q, k, v, o, s, pool
     torch.cuda.empty_cache()
-    return dict(workload="varlen 64 seqs len~U[1K,32K] (T=%d), H=32, d=128, bf16, 32 resumed from fp32 states" % T,
-                tokens_per_s=T * dist.world / (ms_step / 1e3), ms_per_step=ms_step, hbm_gbs=gbs,
-                frac=gbs / pk["hbm"], tflops_rec=flops_rec(T * H, d) / (ms_step / 1e3) / 1e12, steps=n)
+    return res
 
 
-def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0):
+def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0, cpu=False):
     import long_context_linear_b200 as la
     import synth
     c = PREFILL8K
@@ -477,13 +496,45 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0):
     ms_step = total_ms / n
     byts = prefill_bytes(B, H, N, d)
     gbs = byts / (ms_step / 1e3) / 1e9
+    res = dict(workload=f"prefill B=4 H=32 N=8192 d={d} bf16, feature map {phi}",
+               tokens_per_s=B * N * dist.world / (ms_step / 1e3),
+               ms_per_step=ms_step, hbm_gbs=gbs, frac=gbs / pk["hbm"],
+               tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
+               l2="inputs (%.0f MiB) larger than L2" % (3 * B * H * N * d * 2 / 2**20))
+    if cpu:
+        units = torch.tensor(synth.choose(B * H, CPU_8K_UNITS, seed=1), device=dev)
+        qs, ks, vs = (x.view(B * H, N, d)[units].cpu() for x in (q, k, v))
+        res["cpu_baseline"] = oracle_dense_baseline(qs, ks, vs, H, f"{CPU_8K_UNITS} of the {B * H} (batch, head) "
+                                                    f"units of B=4 H=32 N=8192 d={d}, all tokens")
     del q, k, v, o, s, ws
     torch.cuda.empty_cache()
-    return dict(workload=f"prefill B=4 H=32 N=8192 d={d} bf16, feature map {phi}",
-                tokens_per_s=B * N * dist.world / (ms_step / 1e3),
-                ms_per_step=ms_step, hbm_gbs=gbs, frac=gbs / pk["hbm"],
-                tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
-                l2="inputs (%.0f MiB) larger than L2" % (3 * B * H * N * d * 2 / 2**20))
+    return res
+
+
+def run_config1(args, dist: Dist, pk, cpu=False):
+    """The fp32 correctness configuration, B=1, H=2, N=256, d=64, chunk 64, zero
+    initial state (FFMA path): a latency-bound call, timed back to back."""
+    import long_context_linear_b200 as la
+    import synth
+    B, H, N, d = 1, 2, 256, 64
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = synth.dense(B, H, N, d, "fp32", seed=1 + dist.rank, device=dev)
+    o = torch.empty_like(v)
+    s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = 200
+    total_ms, _ = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, chunk=64), n,
+                                 max(3, args.warmup), dist, stream)
+    ms_step = dist.max(total_ms) / n
+    res = dict(workload="prefill B=1 H=2 N=256 d=64 fp32, chunk 64, zero initial state (FFMA path)",
+               us_per_step=ms_step * 1e3, tokens_per_s=B * N * dist.world / (ms_step / 1e3),
+               tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
+               l2="inputs (256 KiB) stay in L2: a latency figure")
+    if cpu:
+        res["cpu_baseline"] = oracle_dense_baseline(q.cpu(), k.cpu(), v.cpu(), 1, "the whole workload", reps=50)
+    del q, k, v, o, s
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_varlen_few(args, dist: Dist, pk):
@@ -675,6 +726,90 @@ def cpu_baseline_line(budget_s=12.0):
                        f"N=131072 d=128 workload ({dt:.1f} s); value in headline tokens (64 heads each)")
 
 
+CPU_DECODE_UNITS = 256   # (sequence, head) units of the decode batch the oracle follows over all steps
+CPU_VARLEN_SEQS = 6      # sequences (all 32 heads) of the packed batch
+CPU_8K_UNITS = 16        # (batch, head) units of the 8K prefill
+
+
+def oracle_dense_baseline(q, k, v, heads_per_token, what, reps=1):
+    """The oracle's recurrence on dense host tensors [U, N, d] (or [B, H, N, d]);
+    value in workload tokens/s (a token carries ``heads_per_token`` heads)."""
+    import oracle
+    oracle.build()
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.recurrent(qd, kd, vd)
+    dt = (time.perf_counter() - t0) / reps
+    th = qd.size / qd.shape[-1]
+    return dict(value=th / heads_per_token / dt, unit="tokens/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"fp64 recurrence on {what} ({dt * 1e3:.1f} ms per pass)")
+
+
+def oracle_decode_baseline(S, q, k, v, H):
+    """The oracle's decode step over all steps of a sample of units: S [U, d, d],
+    q, k, v [steps, U, d]; value in decode tokens/s (a token carries H heads)."""
+    import oracle
+    oracle.build()
+    Sd = S.double().numpy()
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    steps, U = qd.shape[0], qd.shape[1]
+    t0 = time.perf_counter()
+    for t in range(steps):
+        _, Sd = oracle.decode(qd[t], kd[t], vd[t], Sd)
+    dt = time.perf_counter() - t0
+    return dict(value=U * steps / H / dt, unit="tokens/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"fp64 decode of {U} of the 16384 (sequence, head) units over all {steps} steps "
+                       f"({dt:.1f} s); value in 64-head tokens")
+
+
+def oracle_varlen_baseline(parts, init, pool):
+    """The oracle's packed recurrence on a sample of whole sequences (all heads),
+    their resumed states included; value in packed tokens/s."""
+    import oracle
+    import synth
+    oracle.build()
+    cu = synth.cu_seqlens([p[0].shape[0] for p in parts])
+    q, k, v = (torch.cat([p[j] for p in parts]).double().numpy() for j in range(3))
+    idx = torch.tensor(init, dtype=torch.int32)
+    t0 = time.perf_counter()
+    oracle.varlen(q, k, v, cu, pool, idx)
+    dt = time.perf_counter() - t0
+    return dict(value=q.shape[0] / dt, unit="tokens/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"fp64 recurrence on {len(parts)} of the 64 sequences ({q.shape[0]} tokens, all 32 heads, "
+                       f"{sum(i >= 0 for i in init)} resumed; {dt:.1f} s)")
+
+
+def _r(x, n=4):
+    """Rounded to n significant digits (short JSON)."""
+    if x is None or isinstance(x, str):
+        return x
+    return float(f"{x:.{n}g}")
+
+
+def summary_line(extras):
+    """Compact per-config figures for the end of the headline line."""
+    out = {}
+
+    def pick(key, name, fields):
+        e = extras.get(key)
+        if not e:
+            return
+        r = {f: _r(e.get(f)) for f in fields if e.get(f) is not None}
+        cb = e.get("cpu_baseline")
+        if cb:
+            r["cpu_tokens_per_s"] = _r(cb["value"])
+            r["cpu_cores"] = cb["cores"]
+        out[name] = r
+
+    pick("decode", "decode_fp32_state", ("hbm_gbs", "frac", "ms_per_step", "tokens_per_s"))
+    pick("varlen", "varlen_resume", ("tokens_per_s", "ms_per_step", "hbm_gbs", "frac"))
+    pick("prefill_8k", "prefill_8k", ("tokens_per_s", "ms_per_step", "hbm_gbs", "frac"))
+    pick("config1_fp32", "config1_fp32", ("us_per_step", "tokens_per_s", "tflops_rec"))
+    pick("backward_8k", "backward_8k", ("ms_per_step", "hbm_gbs", "frac"))
+    return out
+
+
 def reference_arm(args, dist: Dist):
     if dist.rank != 0:
         return 0
@@ -729,26 +864,26 @@ def main():
         head, _ = run_headline(args, dist, pk, sampler)
         head["clocks"]["remeasured_after"] = dict(reasons=first.get("reasons"), sm_mhz=first.get("sm_mhz"))
     extras = {}
+    cpu_ok = dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline
     if not args.no_extras:
-        extras["decode"] = run_decode(args, dist, pk)
+        extras["config1_fp32"] = run_config1(args, dist, pk, cpu_ok)
+        extras["decode"] = run_decode(args, dist, pk, cpu=cpu_ok)
         # state stored in bf16 / fp16, updated in fp32 (the low-precision storage study)
         extras["decode_bf16_state"] = run_decode(args, dist, pk, torch.bfloat16)
         extras["decode_fp16_state"] = run_decode(args, dist, pk, torch.float16)
         extras["decode_fp8_e4m3_state"] = run_decode(args, dist, pk, torch.float8_e4m3fn)
         extras["decode_small_graph"] = run_decode_small_graph(args, dist, pk)
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
-        extras["varlen"] = run_varlen(args, dist, pk)
+        extras["varlen"] = run_varlen(args, dist, pk, cpu_ok)
         extras["varlen_few_long"] = run_varlen_few(args, dist, pk)
-        extras["prefill_8k"] = run_prefill8k(args, dist, pk)
+        extras["prefill_8k"] = run_prefill8k(args, dist, pk, cpu=cpu_ok)
         extras["prefill_8k_elu1"] = run_prefill8k(args, dist, pk, "elu1")
         extras["prefill_8k_relu"] = run_prefill8k(args, dist, pk, "relu")
         extras["prefill_8k_d64"] = run_prefill8k(args, dist, pk, d=64)
         extras["few_heads"] = run_few_heads(args, dist, pk)
         extras["few_heads_fp32"] = run_few_heads(args, dist, pk, "fp32")
         extras["backward_8k"] = run_backward(args, dist, pk)
-    cpu = None
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_line()
+    cpu = cpu_baseline_line() if cpu_ok else None
     if dist.rank == 0:
         d = HEADLINE["d"]
         peak_note = "of measured" if pk["source"] == "measured" else "of fallback"
@@ -774,7 +909,11 @@ def main():
                         peak_tflops_burst=pk["bf16"], frac_rec_of_burst=head["tflops_rec"] / pk["bf16"],
                         peak_source=peak_note),
             e2e=head["e2e"], gpu_launches=head["launches"], clocks=head["clocks"], cpu_baseline=cpu,
-            extras=extras)
+            summary=summary_line(extras))
+        # the detailed figures of every other workload on a line of their own,
+        # then the headline, whose compact summary closes the output
+        if extras:
+            print(json.dumps(dict(bench_extras=extras)), flush=True)
         print(json.dumps(line), flush=True)
     dist.close()
     return 0

@@ -317,9 +317,16 @@ LA_API la_status la_selftest_wait_timeout(int timeout_us, la_stream_t stream);
  *    without ordering between them) race on it: order them on one stream.
  *  - The first call on each device performs a one-time set-up on the host
  *    (it looks up the device address of the scratch array for the current
- *    device); make that first call before any stream capture.
- * Everything else (arguments, layouts, results, errors) is as for
- * la_prefill_varlen.
+ *    device); make that first call before any stream capture.  The set-up is
+ *    redone when the device's context has changed since (after
+ *    cudaDeviceReset, for instance).
+ *  - Without a workspace the call never takes the segment split or the
+ *    separate feature-map pass of la_prefill_varlen_ex (there is no room for
+ *    their states), and the feature map is the identity.  Batches of a few
+ *    long sequences therefore run unsplit, on fewer SMs and slower than
+ *    la_prefill_varlen with the workspace it asks for; the results are the
+ *    same within the parity tolerances.
+ * Everything else (arguments, layouts, errors) is as for la_prefill_varlen.
  */
 #define LA_NOALLOC_MAX_SEQS 4096
 LA_API la_status la_prefill_varlen_noalloc(const void* q, const void* k, const void* v, void* o,

@@ -191,6 +191,41 @@ def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: to
     return dq, dk, dv, ds0
 
 
+def _check_packed(q, k, v, cu_seqlens, state_pool, init_idx, out, s_out):
+    """Device, dtype, contiguity and shape checks of a packed ragged batch;
+    returns (T, H, dk, dv, n_seq, n_pool).  Run before any launch, so that a
+    wrongly sized buffer never reaches a kernel."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, q.device)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k must be [T, H, dk] and v [T, H, dv]")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be [n_seq + 1]")
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n_seq = cu_seqlens.numel() - 1
+    if out is not None:
+        _need(out, "out", q.dtype, q.device)
+        if tuple(out.shape) != (T, H, dv):
+            raise ValueError(f"out must be [T, H, dv] = {(T, H, dv)}, got {tuple(out.shape)}")
+    n_pool = 0
+    if state_pool is not None:
+        _need(state_pool, "state_pool", torch.float32, q.device)
+        if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (H, dk, dv):
+            raise ValueError("state_pool must be [n_pool, H, dk, dv]")
+        n_pool = state_pool.shape[0]
+    if init_idx is not None:
+        _need(init_idx, "init_idx", torch.int32, q.device)
+        if init_idx.numel() != n_seq:
+            raise ValueError("init_idx must have n_seq entries")
+    if s_out is not None:
+        _need(s_out, "s_out", torch.float32, q.device)
+        if tuple(s_out.shape) != (n_seq, H, dk, dv):
+            raise ValueError(f"s_out must be [n_seq, H, dk, dv] = {(n_seq, H, dk, dv)}, got {tuple(s_out.shape)}")
+    return T, H, dk, dv, n_seq, n_pool
+
+
 def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                    state_pool: Optional[torch.Tensor] = None, init_idx: Optional[torch.Tensor] = None, *,
                    chunk: int = 0, out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None,
@@ -201,32 +236,12 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     Sequence n starts from state_pool[init_idx[n]] when init_idx[n] >= 0;
     phi is the feature map on q and k.  Returns (O [T, H, d], S [n_seq, H, d, d]).
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, q.dtype, q.device)
-    _need(cu_seqlens, "cu_seqlens", torch.int32, q.device)
-    if q.dim() != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
-        raise ValueError("q, k must be [T, H, dk] and v [T, H, dv]")
-    T, H, dk = q.shape
-    dv = v.shape[-1]
-    n_seq = cu_seqlens.numel() - 1
+    T, H, dk, dv, n_seq, n_pool = _check_packed(q, k, v, cu_seqlens, state_pool, init_idx, out, s_out)
     dt = _dtype_code(q)
     if out is None:
         out = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
-    _need(out, "out", q.dtype, q.device)
-    n_pool = 0
-    if state_pool is not None:
-        _need(state_pool, "state_pool", torch.float32, q.device)
-        n_pool = state_pool.shape[0]
-        if tuple(state_pool.shape[1:]) != (H, dk, dv):
-            raise ValueError("state_pool must be [n_pool, H, dk, dv]")
-    if init_idx is not None:
-        _need(init_idx, "init_idx", torch.int32, q.device)
-        if init_idx.numel() != n_seq:
-            raise ValueError("init_idx must have n_seq entries")
     if s_out is None and return_state:
         s_out = torch.empty((max(n_seq, 0), H, dk, dv), dtype=torch.float32, device=q.device)
-    if s_out is not None:
-        _need(s_out, "s_out", torch.float32, q.device)
     need = int(lib.la_prefill_varlen_workspace_size_ex(n_seq, T, H, dk, dv, dt, _phi_code(phi)))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -246,21 +261,14 @@ def prefill_varlen_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu
 
     The caller passes every output buffer; the library uses its built-in
     scratch (at most ``_abi.NOALLOC_MAX_SEQS`` sequences per call) instead of a
-    workspace.  Calls share that scratch: order them on one stream.
+    workspace.  Calls share that scratch: order them on one stream.  With no
+    workspace the call never cuts sequences into segments, so batches of a few
+    long sequences run one CTA per (sequence, head, value slice); the feature
+    map is the identity.
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, n, q.dtype, q.device)
-    _need(cu_seqlens, "cu_seqlens", torch.int32, q.device)
-    T, H, dk = q.shape
-    dv = v.shape[-1]
-    n_seq = cu_seqlens.numel() - 1
-    n_pool = 0 if state_pool is None else state_pool.shape[0]
-    if state_pool is not None:
-        _need(state_pool, "state_pool", torch.float32, q.device)
-    if init_idx is not None:
-        _need(init_idx, "init_idx", torch.int32, q.device)
-    if s_out is not None:
-        _need(s_out, "s_out", torch.float32, q.device)
+    if out is None:
+        raise ValueError("out is required: this call allocates nothing")
+    T, H, dk, dv, n_seq, n_pool = _check_packed(q, k, v, cu_seqlens, state_pool, init_idx, out, s_out)
     with torch.cuda.device(q.device):
         _abi.check(lib.la_prefill_varlen_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq, T,
                                                  _ptr(state_pool), n_pool, _ptr(init_idx), _ptr(s_out), H, dk, dv,

@@ -62,6 +62,7 @@ struct DeviceInfo {
     int sms = 0;
     int* status = nullptr;       // device address of g_status_word
     bool attrs_set = false;
+    unsigned long long ctx = 0;  // id of the context the set-up above was made in
     // copy streams of la_prefill_host, created on first use and kept for the
     // life of the process (like a library handle)
     cudaStream_t h2d = nullptr, d2h = nullptr;
@@ -88,6 +89,34 @@ cudaError_t set_simt_attrs() {
                                 simt::smem_bytes<64, 32>());
 }
 
+// Unique id of the calling thread's current CUDA context, 0 when none is
+// current.  Device addresses and function attributes belong to a context: one
+// destroyed and re-created (cudaDeviceReset) gets a new id, so per-device
+// set-up cached under the old id is redone.
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+PFN_ctx_get_current g_ctx_current = nullptr;
+PFN_ctx_get_id g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+unsigned long long current_ctx_id() {
+    std::call_once(g_ctx_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<PFN_ctx_get_current>(fn);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_id = reinterpret_cast<PFN_ctx_get_id>(fn);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!g_ctx_current || !g_ctx_id || g_ctx_current(&c) != CUDA_SUCCESS || !c || g_ctx_id(c, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 la_status device_info(DeviceInfo** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -95,6 +124,9 @@ la_status device_info(DeviceInfo** out) {
     if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device index %d out of range", dev);
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DeviceInfo& d = g_dev[dev];
+    // set-up made in another context (one that is gone, or none is current on
+    // this thread yet): redo it
+    if (d.attrs_set && current_ctx_id() != d.ctx) d.attrs_set = false;
     if (!d.attrs_set) {
         int major = 0;
         if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
@@ -116,6 +148,9 @@ la_status device_info(DeviceInfo** out) {
                 return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
         if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
+        const unsigned long long id = current_ctx_id();
+        if (id != d.ctx) d.h2d = d.d2h = nullptr;  // copy streams of a context that is gone
+        d.ctx = id;
         d.attrs_set = true;
     }
     *out = &d;
@@ -887,21 +922,24 @@ la_status la_decode_commit(const void* k, const void* v, float* S, const int32_t
 namespace lcl {
 namespace {
 int* g_noalloc_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {0};
 std::mutex g_noalloc_mu;
 
-// One-time per-device set-up: the device address of g_noalloc_order for the
-// current device.
+// Per-device set-up: the device address of g_noalloc_order for the current
+// device, looked up once per context (again after the context was destroyed
+// and re-created, e.g. by cudaDeviceReset, whose old address is stale).
 la_status noalloc_scratch(int** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device index %d out of range", dev);
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_ptr[dev] || current_ctx_id() != g_noalloc_ctx[dev]) {
         void* ptr = nullptr;
         if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_order)) != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
         g_noalloc_ptr[dev] = static_cast<int*>(ptr);
+        g_noalloc_ctx[dev] = current_ctx_id();
     }
     *out = g_noalloc_ptr[dev];
     return LA_OK;

@@ -46,3 +46,35 @@ def test_flop_counts(bench):
 def test_weak_scaling_rate(bench):
     # 131072 tokens per rank on 4 ranks in 2 ms (the slowest rank) -> 262.144 M tokens/s
     assert bench.weak_scaling_rate(131072, 4, 2.0) == pytest.approx(262.144e6)
+
+
+def test_summary_line_is_compact_and_complete(bench):
+    cb = dict(value=1.0e4, unit="tokens/s", cores=16, kind="oracle", sample="s" * 200)
+    ex = dict(decode=dict(hbm_gbs=6265.1234, frac=0.957123, ms_per_step=0.345123, tokens_per_s=741234.5,
+                          workload="w" * 100, cpu_baseline=cb),
+              varlen=dict(tokens_per_s=1.1e8, ms_per_step=9.18, hbm_gbs=4012.3, frac=0.61, cpu_baseline=cb),
+              prefill_8k=dict(tokens_per_s=1.2e8, ms_per_step=0.27, hbm_gbs=3955.4, frac=0.60, cpu_baseline=cb),
+              config1_fp32=dict(us_per_step=48.1, tokens_per_s=5.3e6, tflops_rec=0.02, cpu_baseline=cb),
+              backward_8k=dict(ms_per_step=0.69, hbm_gbs=2712.0, frac=0.41))
+    import json
+    s = bench.summary_line(ex)
+    assert set(s) == {"decode_fp32_state", "varlen_resume", "prefill_8k", "config1_fp32", "backward_8k"}
+    assert s["decode_fp32_state"]["hbm_gbs"] == 6265.0 and s["decode_fp32_state"]["cpu_cores"] == 16
+    assert "workload" not in s["decode_fp32_state"]       # long strings stay on the extras line
+    assert len(json.dumps(dict(summary=s))) < 1000       # fits the tail of the output a driver keeps
+
+
+def test_oracle_baselines_on_tiny_samples(bench):
+    import torch
+    import synth
+    q, k, v = synth.dense(2, 3, 64, 64, "fp32", seed=1)
+    r = bench.oracle_dense_baseline(q, k, v, 3, "tiny", reps=2)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    S = torch.zeros(4, 64, 64)
+    qs, ks, vs = synth.qkv((5, 4, 64), 64, "bf16", seed=2)
+    r = bench.oracle_decode_baseline(S, qs, ks, vs, 2)
+    assert r["value"] > 0 and "4 of the 16384" in r["sample"]
+    parts = [tuple(x for x in synth.qkv((n, 2, 64), 64, "bf16", seed=n)) for n in (10, 7)]
+    pool = torch.zeros(1, 2, 64, 64)
+    r = bench.oracle_varlen_baseline(parts, [0, -1], pool)
+    assert r["value"] > 0 and "17 tokens" in r["sample"] and "1 resumed" in r["sample"]

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import synth
-from tests.parity import assert_out, assert_state
+from tests.parity import assert_out, assert_state, assert_varlen_out
 
 pytestmark = pytest.mark.gpu
 
@@ -90,7 +90,7 @@ def test_varlen_with_phi(la, oracle_mod, phi):
     torch.cuda.synchronize()
     assert la.device_status() == 0
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, init, phi=phi)
-    assert_out(o.cpu()[None], ro[None], torch.bfloat16, 1)
+    assert_varlen_out(o.cpu(), ro, cu, torch.bfloat16)
     assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])
 
 
@@ -232,5 +232,5 @@ def test_varlen_with_phi_and_segments(la, oracle_mod, monkeypatch, phi):
     torch.cuda.synchronize()
     assert la.device_status() == 0
     ro, rs = oracle_mod.varlen(q, k, v, cu, phi=phi)
-    assert_out(o.cpu()[None], ro[None], torch.bfloat16, 1)
+    assert_varlen_out(o.cpu(), ro, cu, torch.bfloat16)
     assert_state(s.cpu(), rs, 2, tol=TC_STATE_TOL[phi])

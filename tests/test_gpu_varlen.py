@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import synth
-from tests.parity import assert_guard_intact, assert_out, assert_state, guarded, to64
+from tests.parity import assert_guard_intact, assert_out, assert_state, assert_varlen_out, guarded, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -55,11 +55,7 @@ def test_varlen_matches_oracle(la, oracle_mod, lens, dtype, d):
     o, s = _run(la, cu, q, k, v, pool, idx)
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
     dt = synth.torch_dtype(dtype)
-    # per (sequence, head) unit: compare each sequence's rows separately
-    for n in range(len(lens)):
-        a, b = int(cu[n]), int(cu[n + 1])
-        if b > a:
-            assert_out(o[a:b].transpose(0, 1), ro[a:b].transpose(1, 0, 2), dt, 1)
+    assert_varlen_out(o, ro, cu, dt)
     assert_state(s, rs, 2)
 
 
@@ -110,7 +106,7 @@ def test_varlen_many_short_sequences(la, oracle_mod, n_seq):
     cu, q, k, v, pool, idx = _case(lens, 2, 128, "bf16", seed=9, n_pool=3, resume=resume)
     o, s = _run(la, cu, q, k, v, pool, idx)
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
-    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_varlen_out(o, ro, cu, torch.bfloat16)
     assert_state(s, rs, 2)
 
 
@@ -126,7 +122,7 @@ def test_varlen_segments_match_oracle(la, oracle_mod, monkeypatch, segments, d):
     cu, q, k, v, pool, idx = _case(lens, 3, d, "bf16", seed=61, n_pool=2, resume=[0, 1, -1, 1, -1, 0])
     o, s = _run(la, cu, q, k, v, pool, idx)
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
-    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_varlen_out(o, ro, cu, torch.bfloat16)
     assert_state(s, rs, 2)
 
 
@@ -138,7 +134,7 @@ def test_varlen_segments_automatic(la, oracle_mod):
     assert la.prefill_varlen_workspace_size(2, sum(lens), 2, 128, torch.bfloat16) > 4 * 256
     o, s = _run(la, cu, q, k, v, pool, idx)
     ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
-    assert_out(o[None], ro[None], torch.bfloat16, 1)
+    assert_varlen_out(o, ro, cu, torch.bfloat16)
     assert_state(s, rs, 2)
 
 

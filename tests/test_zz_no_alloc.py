@@ -5,8 +5,10 @@ framework that owns all device memory, or a serving loop where cudaMalloc is
 not allowed).  For them the library offers a variant of la_prefill_varlen
 that uses a scratch array built into the library instead of a caller-provided
 workspace.  This file checks, through the C ABI, that two calls in a row give
-the same results as the workspace-based entry point, and that batches larger
-than the built-in scratch are refused.  It is collected last on purpose.
+the same results as the workspace-based entry point and as the fp64 oracle,
+for both input types and both head sizes, that batches larger than the
+built-in scratch are refused, and that the Python wrapper checks its buffers'
+shapes before it launches anything.  It is collected last on purpose.
 """
 import ctypes
 
@@ -14,7 +16,7 @@ import pytest
 import torch
 
 import synth
-from tests.parity import assert_out, assert_state, to64
+from tests.parity import assert_state, assert_varlen_out, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -25,13 +27,13 @@ def la():
     return la
 
 
-def _batch(lens, H, d, seed):
+def _batch(lens, H, d, dtype, seed):
     cu = synth.cu_seqlens(lens)
     T = int(cu[-1])
-    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=seed)
+    q, k, v = synth.qkv((T, H, d), d, dtype, seed=seed)
     pool = synth.outer_product_state(2 * H, d, d, [300] * (2 * H), seed=seed + 1).view(2, H, d, d)
     idx = torch.tensor([(i % 3) - 1 for i in range(len(lens))], dtype=torch.int32)
-    return [x.cuda() for x in (cu, q, k, v, pool, idx)]
+    return cu, q, k, v, pool, idx
 
 
 def _noalloc(la, cu, q, k, v, pool, idx):
@@ -39,27 +41,65 @@ def _noalloc(la, cu, q, k, v, pool, idx):
     n = cu.numel() - 1
     o = torch.full_like(v, float("nan"))
     s = torch.full((n, H, d, d), float("nan"), dtype=torch.float32, device=q.device)
+    dt = 0 if q.dtype == torch.bfloat16 else 1
     st = la.lib.la_prefill_varlen_noalloc(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), cu.data_ptr(), n, T, pool.data_ptr(),
-        pool.shape[0], idx.data_ptr(), s.data_ptr(), H, d, d, 0, 0,
+        pool.shape[0], idx.data_ptr(), s.data_ptr(), H, d, d, dt, 0,
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, la.lib.la_last_error()
     return o, s
 
 
-def test_noalloc_matches_workspace_entry_point_twice(la):
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("fp32", 128), ("fp32", 64)])
+def test_noalloc_matches_workspace_entry_point_and_oracle_twice(la, oracle_mod, dtype, d):
     # two different batches in a row: the second call must not depend on what
     # the first one left in the shared scratch
+    dt = synth.torch_dtype(dtype)
     for lens, seed in (([700, 1, 0, 129, 2048, 77], 11), ([5, 300, 128, 1000], 12)):
-        cu, q, k, v, pool, idx = _batch(lens, 3, 128, seed)
-        o_ref, s_ref = la.prefill_varlen(q, k, v, cu, pool, idx)
-        o, s = _noalloc(la, cu, q, k, v, pool, idx)
+        cu, q, k, v, pool, idx = _batch(lens, 3, d, dtype, seed + d)
+        dev = [x.cuda() for x in (cu, q, k, v, pool, idx)]
+        o_ref, s_ref = la.prefill_varlen(*dev)
+        o, s = _noalloc(la, *dev)
         torch.cuda.synchronize()
-        for n in range(len(lens)):
-            a, b = int(cu[n]), int(cu[n + 1])
-            if b > a:
-                assert_out(o[a:b].transpose(0, 1).cpu(), to64(o_ref[a:b].transpose(0, 1)), torch.bfloat16, 1)
-        assert_state(s.cpu(), to64(s_ref), 2)
+        assert_varlen_out(o.cpu(), to64(o_ref), cu, dt)
+        assert_state(s.cpu(), to64(s_ref), 2, tol=1e-5)
+        ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+        assert_varlen_out(o.cpu(), ro, cu, dt)
+        assert_state(s.cpu(), rs, 2)
+    assert la.device_status() == 0
+
+
+def test_noalloc_python_wrapper(la, oracle_mod):
+    cu, q, k, v, pool, idx = _batch([40, 0, 300], 2, 128, "bf16", seed=21)
+    dev = [x.cuda() for x in (cu, q, k, v, pool, idx)]
+    out = torch.empty_like(dev[3])
+    s_out = torch.empty(3, 2, 128, 128, dtype=torch.float32, device="cuda")
+    la.prefill_varlen_noalloc(dev[1], dev[2], dev[3], dev[0], dev[4], dev[5], out=out, s_out=s_out)
+    torch.cuda.synchronize()
+    ro, rs = oracle_mod.varlen(q, k, v, cu, pool, idx)
+    assert_varlen_out(out.cpu(), ro, cu, torch.bfloat16)
+    assert_state(s_out.cpu(), rs, 2)
+
+
+def test_noalloc_python_wrapper_rejects_wrong_shapes(la):
+    cu, q, k, v, pool, idx = (x.cuda() for x in _batch([40, 9], 2, 128, "bf16", seed=22))
+    T, H, d = q.shape
+    good_out = torch.empty_like(v)
+    cases = [
+        dict(out=torch.empty(T - 1, H, d, dtype=q.dtype, device="cuda")),           # out too short
+        dict(out=good_out, s_out=torch.empty(1, H, d, d, device="cuda")),           # s_out for 1 of 2 sequences
+        dict(out=good_out, state_pool=pool[:, :1].contiguous()),                    # pool with 1 of 2 heads
+        dict(out=good_out, init_idx=idx[:1].contiguous()),                          # init_idx too short
+    ]
+    for extra in cases:
+        args = dict(state_pool=pool, init_idx=idx)
+        args.update(extra)
+        sp, ii = args.pop("state_pool"), args.pop("init_idx")
+        with pytest.raises(ValueError):
+            la.prefill_varlen_noalloc(q, k, v, cu, sp, ii, **args)
+    with pytest.raises(ValueError):
+        la.prefill_varlen_noalloc(q, k, v[:, :, :64].contiguous(), cu, out=good_out)
+    torch.cuda.synchronize()
     assert la.device_status() == 0
 
 
