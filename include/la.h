@@ -101,9 +101,10 @@ LA_API int la_version(void);
  *   v, o : [B, H, N, d]  dtype `dt`; o is written
  *   s0   : [B, H, d, d]  fp32 state before token 1, or NULL for zero
  *   s_out: [B, H, d, d]  fp32 state after token N, or NULL (not written)
- *   chunk: tile length C (0 = library choice).  Tensor-core path: 128;
- *          FFMA path: 32 or 64 (default 64).  C does not change the result
- *          beyond rounding.
+ *   chunk: tile length C (0 = library choice).  Tensor-core path (bf16):
+ *          128; FFMA path: 32 or 64 (default 64), for fp32 and also for bf16
+ *          when a bf16 call asks for 32 or 64.  C does not change the result
+ *          beyond rounding; other values return LA_ERR_UNSUPPORTED.
  *   workspace/ws_bytes: scratch of at least la_prefill_workspace_size(...)
  *          bytes, 16-byte aligned (may be NULL when that size is 0).  The size
  *          is non-zero when B*H units are too few to fill the GPU and N is

@@ -20,6 +20,7 @@
 #include "la.h"
 #include "sm100.cuh"
 #include "prefill_tc.cuh"
+#include "prefill_wide.cuh"
 #include "prefill_simt.cuh"
 #include "decode.cuh"
 #include "varlen_order.cuh"
@@ -146,6 +147,12 @@ la_status device_info(DeviceInfo** out) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES)) !=
                 cudaSuccess)
                 return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
+        const void* wide_kernels[2] = {reinterpret_cast<const void*>(tcw::prefill_wide_kernel<false>),
+                                       reinterpret_cast<const void*>(tcw::prefill_wide_kernel<true>)};
+        for (const void* kern : wide_kernels)
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tcw::SMEM_BYTES)) !=
+                cudaSuccess)
+                return cuda_fail(e, "cudaFuncSetAttribute(prefill_wide)");
         if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
         const unsigned long long id = current_ctx_id();
@@ -216,8 +223,17 @@ la_status check_chunk(int chunk, bool tcpath) {
     if (chunk == 0) return LA_OK;
     if (tcpath && chunk == tc::C) return LA_OK;
     if (!tcpath && (chunk == 32 || chunk == 64)) return LA_OK;
-    return fail(LA_ERR_UNSUPPORTED, "chunk %d is not available on this path (%s)", chunk,
-                tcpath ? "tensor-core path: 0 or 128" : "FFMA path: 0, 32 or 64");
+    return fail(LA_ERR_UNSUPPORTED,
+                "chunk %d is not available: 0 (library choice), 128 (bf16 on the tensor cores), "
+                "32 or 64 (FFMA kernel, bf16 or fp32)", chunk);
+}
+
+// The tensor-core kernels tile 128 tokens per chunk (one M = 128 tcgen05 tile
+// of rows); a bf16 call that asks for 32- or 64-token chunks runs on the FFMA
+// kernel, which has those tile lengths.  The result does not depend on the
+// chunk length beyond rounding.
+bool tensor_core_path(int d, la_dtype dt, int chunk) {
+    return use_tensor_cores(d, dt) && (chunk == 0 || chunk == tc::C);
 }
 
 la_status after_launch(const char* what) {
@@ -249,6 +265,32 @@ la_status launch_tc(int grid, const CUtensorMap& mq, const CUtensorMap& mk, cons
 
 // (unit, value slice) work items per unit of the tensor-core prefill
 int tc_slices(int d) { return d / tc::DVS; }
+
+// The full-width kernel (one CTA per head over all 128 value columns) once
+// the batch's heads alone fill the GPU, i.e. when the (head, 64-column value
+// slice) items of the value-split kernel would need more than one wave:
+// it forms Q K^T once per head and needs no more CTAs than there are heads.
+// Below that the value split (and, when still under-filled, the segment
+// split) keeps every SM busy.  LA_PREFILL_WIDE=1 / 0 forces it on / off at
+// d = 128 (on: whole sequences, no segment split).
+bool use_wide(long units, int d, const DeviceInfo* di) {
+    if (d != 128) return false;
+    if (const char* e = getenv("LA_PREFILL_WIDE")) {
+        if (e[0] == '1') return true;
+        if (e[0] == '0') return false;
+    }
+    return units * tc_slices(d) > di->sms;
+}
+
+// The full-width kernel: the lean instance unless the feature map, the
+// reverse order or a transposed initial state asks for the general one.
+la_status launch_wide(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
+    const bool general = p.phi != LA_PHI_IDENTITY || p.reverse || p.init_transposed;
+    if (general) tcw::prefill_wide_kernel<true><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    else tcw::prefill_wide_kernel<false><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    return after_launch(what);
+}
 
 template <typename T, int D>
 void launch_simt_d(int cs, int grid, const void* q, const void* k, const void* v, void* o, const simt::Params& sp,
@@ -494,7 +536,7 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     if (N > 0 && (!q || !k || !v || !o)) return fail(LA_ERR_INVALID_ARG, "q, k, v, o must be non-null");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(s0) || !aligned16(s_out))
         return fail(LA_ERR_INVALID_ARG, "all pointers must be 16-byte aligned");
-    const bool tcpath = use_tensor_cores(dk, dt);
+    const bool tcpath = tensor_core_path(dk, dt, chunk);
     if ((s = check_chunk(chunk, tcpath)) != LA_OK) return s;
     DeviceInfo* di;
     if ((s = device_info(&di)) != LA_OK) return s;
@@ -518,12 +560,13 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     p.n_seg = 1;
     p.phi = phi;
     if (N == 0 && !s_out) return LA_OK;
+    const bool wide = use_wide(U, dk, di);
     int seg_len;
-    int P = plan_segments(U, N, tc_slices(dk), di->sms, &seg_len);
+    int P = wide ? 1 : plan_segments(U, N, tc_slices(dk), di->sms, &seg_len);
     p.seg_len = seg_len;
     const size_t ws_need = segment_workspace_bytes(U, P, dk, dv);
-    if (P > 1 && (!workspace || ws_bytes < ws_need || !aligned16(workspace) ||
-                  (long)U * P * nvs > (1L << 30))) {
+    if (wide || (P > 1 && (!workspace || ws_bytes < ws_need || !aligned16(workspace) ||
+                           (long)U * P * nvs > (1L << 30)))) {
         P = 1;  // no room for the segment states: one pass over whole sequences
         p.seg_len = ((N + tc::C - 1) / tc::C) * tc::C;
     }
@@ -571,6 +614,10 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
         p.n_seg = P;
         p.n_items = (int)(U * P * nvs);
         p.seg_init = starts;
+    }
+    if (wide) {
+        p.n_items = (int)U;
+        return launch_wide(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_wide launch");
     }
     const int grid = std::min(p.n_items, di->sms);
     return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc launch");
@@ -662,7 +709,7 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         (reinterpret_cast<uintptr_t>(init_idx) & 3u))
         return fail(LA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned, index arrays 4-byte aligned");
     if ((long)T * H > (1L << 40) || (long)n_seq * H > (1L << 30)) return fail(LA_ERR_INVALID_ARG, "problem too large");
-    const bool tcpath = use_tensor_cores(dk, dt);
+    const bool tcpath = tensor_core_path(dk, dt, chunk);
     if ((s = check_chunk(chunk, tcpath)) != LA_OK) return s;
     const size_t need = varlen_order_bytes(n_seq);
     if (tcpath && (ws_bytes < need || !workspace || !aligned16(workspace)))
@@ -752,8 +799,9 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         off_seg += ws_phi;
     }
     const int nvs = tc_slices(dv);
+    const bool wide = use_wide((long)n_seq * H, dk, di);
     int min_seg;
-    long max_segs = plan_varlen_segments(n_seq, T, H, nvs, di->sms, &min_seg);
+    long max_segs = wide ? 0 : plan_varlen_segments(n_seq, T, H, nvs, di->sms, &min_seg);
     if (max_segs && (ws_bytes < off_seg + varlen_segment_bytes(n_seq, max_segs, H, dk) ||
                      max_segs * H * nvs > (1L << 30)))
         max_segs = 0;  // no room for the segment states: whole sequences
@@ -818,6 +866,10 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
         if ((s = after_launch("varlen segment prefix launch")) != LA_OK) return s;
         p.n_items = (int)(max_segs * H * nvs);
         p.seg_init = starts;
+    }
+    if (wide) {
+        p.n_items = (int)((long)n_seq * H);
+        return launch_wide(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_wide (varlen) launch");
     }
     const int grid = std::min(p.n_items, di->sms);
     return launch_tc(grid, mq, mk, mv, mo, p, st, "prefill_tc (varlen) launch");
@@ -990,8 +1042,9 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
     p.phi = LA_PHI_IDENTITY;
     p.reverse = reverse ? 1 : 0;
     p.init_transposed = init_t ? 1 : 0;
+    const bool wide = use_wide(U, d, di);
     int seg_len;
-    int P = plan_segments(U, N, tc_slices(d), di->sms, &seg_len);
+    int P = wide ? 1 : plan_segments(U, N, tc_slices(d), di->sms, &seg_len);
     if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) ||
                   U * P * nvs > (1L << 30)))
         P = 1;
@@ -1028,6 +1081,10 @@ static la_status tc_dense_pass(const void* q, const void* k, const void* v, void
         p.n_items = (int)(U * P * nvs);
         p.seg_init = starts;
         p.init_transposed = 0;  // the segment starts are in the usual layout
+    }
+    if (wide) {
+        p.n_items = (int)U;
+        return launch_wide(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_wide (backward pass) launch");
     }
     return launch_tc(std::min(p.n_items, di->sms), mq, mk, mv, mo, p, st, "prefill_tc (backward pass) launch");
 }

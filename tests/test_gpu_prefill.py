@@ -194,3 +194,31 @@ def test_tc_d64_integer_inputs_bit_exact(la, oracle_mod):
     ro, rs = oracle_mod.recurrent(q, k, v, s0)
     assert torch.equal(o, torch.from_numpy(ro).to(torch.bfloat16))
     np.testing.assert_array_equal(to64(s), rs)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("chunk", [32, 64])
+def test_bf16_small_chunks_match_oracle(la, oracle_mod, d, chunk):
+    """bf16 with 32- or 64-token chunks runs on the FFMA kernel (the tensor-core
+    tiles are 128 tokens long); the chunk length does not change the result
+    beyond rounding, so the bars are the same."""
+    q, k, v = synth.dense(2, 2, 300, d, "bf16", seed=d + chunk)
+    s0 = _state(2, 2, d, seed=chunk)
+    o, s = _run(la, q, k, v, s0, chunk=chunk)
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o, ro, torch.bfloat16, 2)
+    assert_state(s, rs, 2)
+
+
+def test_bf16_chunk64_varlen_matches_oracle(la, oracle_mod):
+    lens = [300, 0, 1, 129, 64]
+    cu = synth.cu_seqlens(lens)
+    T, H, d = int(cu[-1]), 2, 128
+    q, k, v = synth.qkv((T, H, d), d, "bf16", seed=7)
+    o, s = la.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), chunk=64)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.varlen(q, k, v, cu)
+    from tests.parity import assert_varlen_out
+    assert_varlen_out(o.cpu(), ro, cu, torch.bfloat16)
+    assert_state(s.cpu(), rs, 2)

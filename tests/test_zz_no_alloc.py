@@ -57,9 +57,9 @@ def test_noalloc_matches_workspace_entry_point_and_oracle_twice(la, oracle_mod, 
     dt = synth.torch_dtype(dtype)
     for lens, seed in (([700, 1, 0, 129, 2048, 77], 11), ([5, 300, 128, 1000], 12)):
         cu, q, k, v, pool, idx = _batch(lens, 3, d, dtype, seed + d)
-        dev = [x.cuda() for x in (cu, q, k, v, pool, idx)]
-        o_ref, s_ref = la.prefill_varlen(*dev)
-        o, s = _noalloc(la, *dev)
+        cu_d, q_d, k_d, v_d, pool_d, idx_d = (x.cuda() for x in (cu, q, k, v, pool, idx))
+        o_ref, s_ref = la.prefill_varlen(q_d, k_d, v_d, cu_d, pool_d, idx_d)
+        o, s = _noalloc(la, cu_d, q_d, k_d, v_d, pool_d, idx_d)
         torch.cuda.synchronize()
         assert_varlen_out(o.cpu(), to64(o_ref), cu, dt)
         assert_state(s.cpu(), to64(s_ref), 2, tol=1e-5)
