@@ -49,12 +49,12 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 
 # DRAM traffic of one prefill launch, from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum) of the kernel built from sources with this hash, on
-# the H=16, N=32768 case: 517.10 MB for 16*32768 token-heads.  Traffic grows
+# the H=16, N=32768 case: 517.0 MB for 16*32768 token-heads.  Traffic grows
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "025a97fe7bbf03f1"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.710016e6 + 114.394880e6) / (16 * 32768)
+TRAFFIC_HASH = "1c63d16b44b4bc9e"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.72256e6 + 114.2464e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
