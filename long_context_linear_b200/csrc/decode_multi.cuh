@@ -50,38 +50,51 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float4 y) {
     *reinterpret_cast<uint2*>(dst) = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
 }
 
-// verify, one CTA of D / 2 threads per unit, in two row groups of D / 4:
-// thread (g, c) owns value columns 4c .. 4c + 3 and rows g * D / 2 .. of S_0,
-// which it streams from HBM one 16-byte piece per row (8 rows in flight),
-// updating the q_t S_0 sums of all MB drafts per piece.  q is also stored
+// A piece of S_0: streamed past L1 when one draft group reads it, cached in
+// L1 for the other groups when several do.
+template <bool kOneGroup>
+__device__ __forceinline__ float4 load_s(const float4* p) {
+    if constexpr (kOneGroup) return __ldcs(p);
+    else return __ldg(p);
+}
+
+// verify, one CTA per unit of D / 2 threads per group of DPG drafts (MB / DPG
+// groups, MB = 4, 8, 12 or 16 >= m; drafts past m are zero and not stored).
+// In each draft group, thread (g, c) owns value columns 4c .. 4c + 3 and rows
+// g * D / 2 .. of S_0 in two row groups of D / 4 threads, streams them one
+// 16-byte piece per row (8 rows in flight) and updates the q_t S_0 sums of its
+// DPG drafts per piece (4 DPG accumulators).  Several draft groups read the
+// same pieces (HBM once, L1 or L2 for the others).  q is also stored
 // transposed, draft index fastest, so that four drafts' q_i come in one
-// broadcast load.  Row group 1 hands its partial sums to group 0 through
-// shared memory; group 0 adds them and the intra-draft terms and stores o.
-// MB = 4, 8, 12 or 16 >= m (drafts past m are zero and not stored).  Keeping a
-// second batch of rows in flight per thread was measured slower (its
-// registers cost more occupancy than the overlap gained: m = 16, 0.739 ms
-// against 0.664).
-template <typename T, int D, int MB>
-__global__ void __launch_bounds__(D / 2)
+// broadcast load.  Row group 1 hands its partial sums to row group 0 through
+// shared memory; row group 0 adds them and the intra-draft terms and stores o.
+// Measured at B=256, H=64 (ms): one group for m <= 12; at m = 16 one group of
+// 16 (161 registers, 12 warps per SM) took 0.59, four groups of 4 took 0.77
+// (the extra state reads go to L2).
+template <typename T, int D, int MB, int DPG>
+__global__ void __launch_bounds__(D / 2 * (MB / DPG))
 verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
               const float* __restrict__ S, int m, int phi) {
-    constexpr int LPR = D / 4;  // threads per row group
-    constexpr int NT = 2 * LPR;
-    constexpr int ROWS = D / 2;  // rows per group
-    constexpr int UNR = 8;       // rows in flight per thread
-    static_assert(ROWS % UNR == 0 && MB % 4 == 0 && MB <= MAX_M, "verify layout");
+    constexpr int LPR = D / 4;     // threads per row group
+    constexpr int NG = 2 * LPR;    // threads per draft group
+    constexpr int NT = NG * (MB / DPG);
+    constexpr int ROWS = D / 2;    // rows per row group
+    constexpr int UNR = 8;         // rows in flight per thread
+    static_assert(ROWS % UNR == 0 && MB % DPG == 0 && DPG % 4 == 0 && MB <= MAX_M, "verify layout");
+    constexpr bool kOne = MB == DPG;
     __shared__ __align__(16) float qT[D][MB];
     __shared__ __align__(16) float qs[MB][D], ks[MB][D], vs[MB][D];
     __shared__ float A[MB][MB];  // A[t][s] = q_t . k_s, s <= t
-    float(*red)[D] = qs;         // group 1's partial sums, once the scores are done with q
+    float(*red)[D] = qs;         // row group 1's partial sums, once the scores are done with q
 
     const long u = blockIdx.x;
-    const int tid = threadIdx.x, g = tid / LPR, c = tid % LPR;
+    const int tid = threadIdx.x, dg = tid / NG, g = (tid % NG) / LPR, c = tid % LPR;
+    const int t0 = DPG * dg;  // this thread's drafts t0 .. t0 + DPG - 1
     // the first rows of S_0 are requested before the drafts are read
     const float4* Sg = reinterpret_cast<const float4*>(S + u * D * D) + (long)g * ROWS * LPR + c;
     float4 x[UNR];
 #pragma unroll
-    for (int j = 0; j < UNR; ++j) x[j] = __ldcs(Sg + (long)j * LPR);
+    for (int j = 0; j < UNR; ++j) x[j] = load_s<kOne>(Sg + (long)j * LPR);
     // the drafts' q, k, v (phi on q and k), zero past m; 16-byte loads
     const long base = u * (long)m * D;
     constexpr int VEC = 16 / (int)sizeof(T);
@@ -129,21 +142,21 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         }
     }
     __syncthreads();  // qs is reused for the partial sums below
-    // q_t S_0 over this group's rows for all MB drafts
-    float4 acc[MB];
+    // q_t S_0 over this row group's rows for the thread's drafts
+    float4 acc[DPG];
 #pragma unroll
-    for (int t = 0; t < MB; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < DPG; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
     for (int r0 = 0; r0 < ROWS; r0 += UNR) {
         if (r0 > 0) {
 #pragma unroll
-            for (int j = 0; j < UNR; ++j) x[j] = __ldcs(Sg + (long)(r0 + j) * LPR);
+            for (int j = 0; j < UNR; ++j) x[j] = load_s<kOne>(Sg + (long)(r0 + j) * LPR);
         }
 #pragma unroll
         for (int j = 0; j < UNR; ++j) {
-            const float* qrow = qT[g * ROWS + r0 + j];
+            const float* qrow = qT[g * ROWS + r0 + j] + t0;
 #pragma unroll
-            for (int t4 = 0; t4 < MB; t4 += 4) {
+            for (int t4 = 0; t4 < DPG; t4 += 4) {
                 const float4 qq = *reinterpret_cast<const float4*>(qrow + t4);
                 const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
@@ -159,15 +172,16 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
     if (g == 1) {
 #pragma unroll
-        for (int t = 0; t < MB; ++t) *reinterpret_cast<float4*>(&red[t][4 * c]) = acc[t];
+        for (int tt = 0; tt < DPG; ++tt) *reinterpret_cast<float4*>(&red[t0 + tt][4 * c]) = acc[tt];
     }
     __syncthreads();
     if (g == 0) {
 #pragma unroll
-        for (int t = 0; t < MB; ++t) {
+        for (int tt = 0; tt < DPG; ++tt) {
+            const int t = t0 + tt;
             if (t < m) {
                 const float4 p = *reinterpret_cast<const float4*>(&red[t][4 * c]);
-                float4 y = make_float4(acc[t].x + p.x, acc[t].y + p.y, acc[t].z + p.z, acc[t].w + p.w);
+                float4 y = make_float4(acc[tt].x + p.x, acc[tt].y + p.y, acc[tt].z + p.z, acc[tt].w + p.w);
                 for (int s = 0; s <= t; ++s) {
                     const float a = A[t][s];
                     const float4 vv = *reinterpret_cast<const float4*>(&vs[s][4 * c]);

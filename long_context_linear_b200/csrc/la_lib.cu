@@ -337,10 +337,11 @@ namespace {
 template <typename T, int D>
 void launch_verify_d(int m, int grid, const T* q, const T* k, const T* v, T* o, const float* S, int phi,
                      cudaStream_t st) {
-    if (m <= 4) dmulti::verify_kernel<T, D, 4><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
-    else if (m <= 8) dmulti::verify_kernel<T, D, 8><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
-    else if (m <= 12) dmulti::verify_kernel<T, D, 12><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
-    else dmulti::verify_kernel<T, D, 16><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    // D / 2 threads per group of drafts: one group up to 12 drafts, two of 8 beyond
+    if (m <= 4) dmulti::verify_kernel<T, D, 4, 4><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else if (m <= 8) dmulti::verify_kernel<T, D, 8, 8><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else if (m <= 12) dmulti::verify_kernel<T, D, 12, 12><<<grid, D / 2, 0, st>>>(q, k, v, o, S, m, phi);
+    else dmulti::verify_kernel<T, D, 16, 8><<<grid, D, 0, st>>>(q, k, v, o, S, m, phi);
 }
 template <typename T>
 void launch_verify(int dk, int m, int grid, const void* q, const void* k, const void* v, void* o, const float* S,
