@@ -23,6 +23,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include "decode.cuh"
+#include "sm100.cuh"
 
 namespace lcl {
 namespace dmulti {
@@ -193,6 +194,166 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
                 store4(o + base + (long)t * D + 4 * c, y);
             }
         }
+    }
+}
+
+// verify on the tensor cores, bf16 q, k, v at d = 128 (fp32 S_0), one CTA of
+// 128 threads per unit.  The inter-draft part is one product per unit,
+//   O^T = bf16(S_0)^T Q^T    (M = 128 value columns, N = 16 drafts, K = 128),
+// with bf16(S_0) as the operand and fp32 accumulation -- the same reading as
+// the prefill's Q S product -- so that the tensor cores, not the FMA pipes,
+// carry the m d^2 work whatever m is.  The threads convert S_0 to bf16 in the
+// MN-major 128B-swizzled layout (row i of S_0 is K-step row i, two 64-column
+// panels), Q (zero past m) to a K-major tile of 16 rows, one thread issues the
+// 8 tcgen05.mma, and thread j reads column j of O^T (16 drafts) from TMEM,
+// adds the intra-draft terms sum_{s <= t} (q_t . k_s) v_s in fp32 and stores.
+// phi(q) and phi(k) are rounded to bf16 (tensor-core operands) for the scores
+// too, as on the tensor-core prefill.
+constexpr int TC_THREADS = 128;
+
+__global__ void __launch_bounds__(TC_THREADS)
+verify_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ o, const float* __restrict__ S,
+                 int m, int phi, int* status) {
+    constexpr int D = 128, MT = 16;                  // value columns, draft rows of the product
+    constexpr int PANEL_S = D * 128;                 // 128 rows x 128 bytes: 64 value columns of bf16(S)
+    constexpr int PANEL_Q = MT * 128;                // 16 rows x 128 bytes: 64 key dims of q
+    __shared__ __align__(1024) uint8_t s_tile[2 * PANEL_S];
+    __shared__ __align__(1024) uint8_t q_tile[2 * PANEL_Q];
+    __shared__ __align__(16) __nv_bfloat16 ksb[MT][D];  // bf16(phi(k)) of the drafts, for the scores
+    __shared__ __align__(16) __nv_bfloat16 qsb[MT][D];  // bf16(phi(q))
+    __shared__ float A[MT][MT];                      // A[t][s] = q_t . k_s, s <= t
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t tmem_holder;
+
+    const long u = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float4* Su = reinterpret_cast<const float4*>(S + u * D * D);
+    // S_0 -> bf16 tile: warp w converts rows w, w + 4, ...; lane c holds columns 4c .. 4c + 3
+    {
+        const int c = lane;
+        const uint32_t panel = static_cast<uint32_t>(c >> 4) * PANEL_S;
+        const uint32_t chunk = static_cast<uint32_t>((c & 15) >> 1), half = static_cast<uint32_t>(c & 1) * 8u;
+        const uint32_t sb = smem_u32(s_tile) + panel + half;
+#pragma unroll 4
+        for (int r0 = 0; r0 < D; r0 += 32) {
+            float4 x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = __ldcs(Su + (long)(r0 + 4 * j + warp) * (D / 4) + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t row = static_cast<uint32_t>(r0 + 4 * j + warp);
+                const uint32_t a = sb + row * 128u + ((chunk ^ (row & 7u)) << 4);
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a), "r"(pack_bf16x2(x[j].x, x[j].y)),
+                             "r"(pack_bf16x2(x[j].z, x[j].w))
+                             : "memory");
+            }
+        }
+    }
+    // the drafts: phi(q) as a K-major bf16 tile and in fp32, phi(k) and v in fp32
+    const long base = u * (long)m * D;
+    for (int e = tid * 8; e < MT * D; e += TC_THREADS * 8) {
+        const int t = e / D, i = e % D;
+        float qv[8], kv[8];
+        if (t < m) {
+            unpack16(*reinterpret_cast<const uint4*>(q + base + e), qv);
+            unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                qv[jj] = apply_phi(qv[jj], phi);
+                kv[jj] = apply_phi(kv[jj], phi);
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) qv[jj] = kv[jj] = 0.f;
+        }
+        const uint4 qp = make_uint4(pack_bf16x2(qv[0], qv[1]), pack_bf16x2(qv[2], qv[3]), pack_bf16x2(qv[4], qv[5]),
+                                    pack_bf16x2(qv[6], qv[7]));
+        *reinterpret_cast<uint4*>(&qsb[t][i]) = qp;
+        *reinterpret_cast<uint4*>(&ksb[t][i]) = make_uint4(pack_bf16x2(kv[0], kv[1]), pack_bf16x2(kv[2], kv[3]),
+                                                           pack_bf16x2(kv[4], kv[5]), pack_bf16x2(kv[6], kv[7]));
+        // the same 8 bf16 of row t, key dims i .. i + 7, as one 16-byte chunk of the K-major tile
+        const uint32_t qa = smem_u32(q_tile) + static_cast<uint32_t>(i >> 6) * PANEL_Q + static_cast<uint32_t>(t) * 128u +
+                            ((static_cast<uint32_t>((i & 63) >> 3) ^ static_cast<uint32_t>(t & 7)) << 4);
+        st_shared_v4(qa, qp.x, qp.y, qp.z, qp.w);
+    }
+    fence_proxy_async_smem();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_holder, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_holder;
+    if (tid == 0) {
+        constexpr uint32_t id = idesc_bf16(128, MT, 1, 0);  // A = bf16(S_0)^T MN-major, B = Q^T K-major
+        const uint64_t da = sw128_desc(smem_u32(s_tile), PANEL_S, 1024);
+        const uint64_t db = sw128_desc(smem_u32(q_tile), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a_step = static_cast<uint64_t>(kk) * (2048u >> 4);
+            const uint64_t b_step = static_cast<uint64_t>((static_cast<uint32_t>(kk >> 2) * PANEL_Q + static_cast<uint32_t>(kk & 3) * 32u) >> 4);
+            mma_ss(tbase, da + a_step, db + b_step, id, kk > 0);
+        }
+        mma_commit(&bar);
+    }
+    // intra-draft scores while the product runs: one warp per pair (t, s), s <= t
+    {
+        int t = 0, s = warp;
+        while (s > t) { s -= t + 1; ++t; }
+        for (; t < m;) {
+            float a = 0.f;
+#pragma unroll
+            for (int i = lane; i < D; i += 32) a = fmaf(__bfloat162float(qsb[t][i]), __bfloat162float(ksb[s][i]), a);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+            if (lane == 0) A[t][s] = a;
+            s += TC_THREADS / 32;
+            while (s > t) { s -= t + 1; ++t; }
+        }
+    }
+    __syncthreads();
+    // O^T column j = tid: 16 drafts from TMEM (lane j), then the intra-draft terms
+    bool ok = true;
+    {
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(&bar, 0)) {
+            if (globaltimer() - t0 > kWaitTimeoutNs) {
+                atomicExch(status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+        }
+    }
+    tc_fence_after();
+    uint32_t r[16];
+    tmem_ld16(tbase + (static_cast<uint32_t>(warp * 32) << 16), r);
+    tmem_wait_ld();
+    if (ok) {
+        const int j = tid;
+        float vj[MT];
+#pragma unroll
+        for (int s = 0; s < MT; ++s) vj[s] = s < m ? __bfloat162float(v[base + (long)s * D + j]) : 0.f;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            if (t < m) {
+                float y = __uint_as_float(r[t]);
+#pragma unroll
+                for (int s = 0; s <= t; ++s) y = fmaf(A[t][s], vj[s], y);
+                o[base + (long)t * D + j] = __float2bfloat16_rn(y);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 32);
     }
 }
 

@@ -919,6 +919,14 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o, f
     return la_decode_step_ex(q, k, v, o, S, B, H, dk, dv, dt, LA_STATE_FP32, LA_PHI_IDENTITY, stream);
 }
 
+// Drafts up to which the FFMA verify kernel is the faster one (measured at
+// B=256, H=64, d=128, bf16, ms, FFMA / tensor cores: m = 1 0.154 / 0.277,
+// m = 4 0.164 / 0.284, m = 8 0.242 / 0.328, m = 12 0.391 / 0.396, m = 16
+// 0.584 / 0.456): the tensor-core kernel has a higher fixed cost per unit
+// (its S_0 load and conversion do not overlap its product), but its cost
+// grows less with m.
+constexpr int kVerifyFfmaMaxM = 12;
+
 la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S, int B, int H,
                            int m, int dk, int dv, la_dtype dt, la_phi phi, la_stream_t stream) {
     g_last_error[0] = 0;
@@ -936,7 +944,16 @@ la_status la_decode_verify(const void* q, const void* k, const void* v, void* o,
     DeviceInfo* di;
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (dt == LA_BF16) launch_verify<__nv_bfloat16>(dk, m, (int)U, q, k, v, o, S, phi, st);
+    // bf16 at d = 128: the q S_0 products on the tensor cores once the drafts
+    // make the FFMA kernel compute-bound (LA_VERIFY_TC=1 / 0 forces it on / off)
+    bool tcv = dt == LA_BF16 && dk == 128 && m > kVerifyFfmaMaxM;
+    if (dt == LA_BF16 && dk == 128)
+        if (const char* e = getenv("LA_VERIFY_TC")) tcv = e[0] == '1';
+    if (tcv)
+        dmulti::verify_tc_kernel<<<(int)U, dmulti::TC_THREADS, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
+            reinterpret_cast<const __nv_bfloat16*>(v), reinterpret_cast<__nv_bfloat16*>(o), S, m, phi, di->status);
+    else if (dt == LA_BF16) launch_verify<__nv_bfloat16>(dk, m, (int)U, q, k, v, o, S, phi, st);
     else launch_verify<float>(dk, m, (int)U, q, k, v, o, S, phi, st);
     return after_launch("decode_verify launch");
 }

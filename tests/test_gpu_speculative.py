@@ -43,6 +43,28 @@ def test_verify_matches_recurrence_over_drafts(la, oracle_mod, m, d, dtype):
     assert_out(o.cpu(), ro, q.dtype, 2)
 
 
+@pytest.mark.parametrize("m", [1, 3, 4, 5, 8, 13, 16])
+@pytest.mark.parametrize("phi", ["identity", "relu", "elu1"])
+def test_verify_tensor_cores_match_recurrence(la, oracle_mod, monkeypatch, m, phi):
+    """bf16 at d = 128 with the q S_0 products on the tensor cores (bf16(S_0)
+    as the operand, fp32 accumulation), forced for every m: the fp64
+    recurrence over the drafts at the bf16 output bars, and the FFMA kernel
+    (fp32 S_0) within the same bars."""
+    B, H, d = 3, 4, 128
+    S, q, k, v = _case(B, H, m, d, "bf16", seed=m * 7 + 1)
+    Sd = S.cuda()
+    monkeypatch.setenv("LA_VERIFY_TC", "1")
+    o_tc = la.decode_verify(q.cuda(), k.cuda(), v.cuda(), Sd, phi=phi)
+    monkeypatch.setenv("LA_VERIFY_TC", "0")
+    o_ff = la.decode_verify(q.cuda(), k.cuda(), v.cuda(), Sd, phi=phi)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    assert torch.equal(Sd.cpu(), S), "verify must not change the state"
+    ro, _ = oracle_mod.recurrent(q, k, v, S, phi=phi)
+    assert_out(o_tc.cpu(), ro, torch.bfloat16, 2)
+    assert_out(o_tc.cpu(), o_ff.cpu().double().numpy(), torch.bfloat16, 2)
+
+
 @pytest.mark.parametrize("m", [1, 4, 16])
 def test_commit_matches_recurrence_over_accepted_prefix(la, oracle_mod, m):
     B, H, d = 5, 3, 128
