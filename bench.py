@@ -407,6 +407,16 @@ def run_speculative(args, dist: Dist, pk, m: int = 4):
 
     total_ms, _ = timed_launches(spec, rounds, max(3, args.warmup), dist, stream)
     ms_spec = dist.max(total_ms) / rounds
+    it[0] = 0
+    o_ver = torch.empty_like(q[0])
+
+    def verify_only():
+        r = it[0] % rounds
+        la.decode_verify(q[r], k[r], v[r], S, out=o_ver)
+        it[0] += 1
+
+    total_ms, _ = timed_launches(verify_only, rounds, max(3, args.warmup), dist, stream)
+    ms_verify = dist.max(total_ms) / rounds
     qs, ks, vs = (x.permute(0, 3, 1, 2, 4).contiguous() for x in (q, k, v))  # [rounds, m, B, H, d]
     it[0] = 0
 
@@ -419,14 +429,17 @@ def run_speculative(args, dist: Dist, pk, m: int = 4):
     total_ms, _ = timed_launches(steps, rounds, max(3, args.warmup), dist, stream)
     ms_steps = dist.max(total_ms) / rounds
     bytes_spec = 3.0 * U * d * d * 4 + 4.0 * U * m * d * 2
-    del S, q, k, v, qs, ks, vs
+    # verify alone: each state read once, q, k, v read and o written
+    bytes_verify = 1.0 * U * d * d * 4 + 4.0 * U * m * d * 2
+    del S, q, k, v, qs, ks, vs, o_ver
     torch.cuda.empty_cache()
     return dict(workload=f"speculative decode B=256 H=64 d=128 bf16, fp32 state, m={m} drafts all accepted",
                 ms_verify_commit=ms_spec, ms_m_decode_steps=ms_steps,
                 tokens_per_s=B * m * dist.world / (ms_spec / 1e3),
                 tokens_per_s_decode_steps=B * m * dist.world / (ms_steps / 1e3),
                 hbm_gbs=bytes_spec / (ms_spec / 1e3) / 1e9, frac=bytes_spec / (ms_spec / 1e3) / 1e9 / pk["hbm"],
-                rounds=rounds)
+                ms_verify=ms_verify, verify_hbm_gbs=bytes_verify / (ms_verify / 1e3) / 1e9,
+                verify_frac=bytes_verify / (ms_verify / 1e3) / 1e9 / pk["hbm"], rounds=rounds)
 
 
 def run_varlen(args, dist: Dist, pk, cpu=False):
@@ -807,6 +820,7 @@ def summary_line(extras):
     pick("prefill_8k", "prefill_8k", ("tokens_per_s", "ms_per_step", "hbm_gbs", "frac"))
     pick("config1_fp32", "config1_fp32", ("us_per_step", "tokens_per_s", "tflops_rec"))
     pick("backward_8k", "backward_8k", ("ms_per_step", "hbm_gbs", "frac"))
+    pick("speculative_m16", "verify_m16", ("ms_verify", "verify_hbm_gbs", "verify_frac"))
     return out
 
 
@@ -874,6 +888,7 @@ def main():
         extras["decode_fp8_e4m3_state"] = run_decode(args, dist, pk, torch.float8_e4m3fn)
         extras["decode_small_graph"] = run_decode_small_graph(args, dist, pk)
         extras["speculative_m4"] = run_speculative(args, dist, pk, 4)
+        extras["speculative_m16"] = run_speculative(args, dist, pk, 16)
         extras["varlen"] = run_varlen(args, dist, pk, cpu_ok)
         extras["varlen_few_long"] = run_varlen_few(args, dist, pk)
         extras["prefill_8k"] = run_prefill8k(args, dist, pk, cpu=cpu_ok)

@@ -197,157 +197,270 @@ verify_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
 }
 
-// verify on the tensor cores, bf16 q, k, v at d = 128 (fp32 S_0), one CTA of
-// 128 threads per unit.  The inter-draft part is one product per unit,
-//   O^T = bf16(S_0)^T Q^T    (M = 128 value columns, N = 16 drafts, K = 128),
-// with bf16(S_0) as the operand and fp32 accumulation -- the same reading as
-// the prefill's Q S product -- so that the tensor cores, not the FMA pipes,
-// carry the m d^2 work whatever m is.  The threads convert S_0 to bf16 in the
-// MN-major 128B-swizzled layout (row i of S_0 is K-step row i, two 64-column
-// panels), Q (zero past m) to a K-major tile of 16 rows, one thread issues the
-// 8 tcgen05.mma, and thread j reads column j of O^T (16 drafts) from TMEM,
-// adds the intra-draft terms sum_{s <= t} (q_t . k_s) v_s in fp32 and stores.
-// phi(q) and phi(k) are rounded to bf16 (tensor-core operands) for the scores
-// too, as on the tensor-core prefill.
-constexpr int TC_THREADS = 128;
+// verify on the tensor cores, persistent: bf16 q, k, v at d = 128, fp32 S_0.
+// One CTA of 128 threads per SM walks the units u = blockIdx.x + n gridDim.x.
+// Thread 32 (lane 0 of warp 1) streams each unit's S_0 (four 32-column fp32 panels by TMA, in the
+// 128-byte swizzle of 32-byte atoms: the layout the tensor cores take for an
+// MN-major tf32 operand) and its v rows (a plain bulk copy) into one of three
+// slots, up to three units ahead of the one being computed, so that about
+// 128 KB of state is in flight per SM and the state never passes through
+// registers; the threads fetch the next unit's q and k rows into registers
+// while the current unit computes.  The inter-draft part is one tcgen05
+// product per unit on the fp32 tiles read as tf32,
+//   O^T = S_0^T Q^T    (M = 128 value columns, N = 16 drafts, K = 128 key dims),
+// with fp32 accumulation in TMEM; meanwhile the threads form the scores
+// A[t][s] = phi(q_t) . phi(k_s) in fp32, and thread j then reads column j of
+// O^T from TMEM, adds sum_{s <= t} A[t][s] v_s[j] and stores o_t[j].
+namespace vtf {
+constexpr int THREADS = 128, D = 128, MT = 16, SLOTS = 3;
+constexpr uint32_t PANEL_S = 128 * 128;                 // 128 key rows x 128 bytes: 32 value columns of fp32
+constexpr uint32_t SLOT_S = 4 * PANEL_S;                // S_0 of one unit, 64 KB
+constexpr uint32_t ROWS = MT * D * 2;                   // room for 16 draft rows of bf16 (v)
+constexpr uint32_t SLOT = SLOT_S + ROWS;
+constexpr uint32_t PANEL_Q = MT * 128;                  // 16 draft rows x 128 bytes: 32 key dims of fp32
+constexpr uint32_t OFF_QT = SLOTS * SLOT;               // phi(q), K-major 128B-swizzled B operand
+constexpr uint32_t OFF_KF = OFF_QT + 4 * PANEL_Q;       // phi(k) row-major fp32, for the scores
+constexpr uint32_t OFF_A = OFF_KF + MT * D * 4;         // A[t][s]
+constexpr uint32_t OFF_BAR = OFF_A + MT * MT * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;    // + alignment slack
+static_assert(SLOT % 1024 == 0 && OFF_QT % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+}  // namespace vtf
 
-__global__ void __launch_bounds__(TC_THREADS)
-verify_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                 const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ o, const float* __restrict__ S,
-                 int m, int phi, int* status) {
-    constexpr int D = 128, MT = 16;                  // value columns, draft rows of the product
-    constexpr int PANEL_S = D * 128;                 // 128 rows x 128 bytes: 64 value columns of bf16(S)
-    constexpr int PANEL_Q = MT * 128;                // 16 rows x 128 bytes: 64 key dims of q
-    __shared__ __align__(1024) uint8_t s_tile[2 * PANEL_S];
-    __shared__ __align__(1024) uint8_t q_tile[2 * PANEL_Q];
-    __shared__ __align__(16) __nv_bfloat16 ksb[MT][D];  // bf16(phi(k)) of the drafts, for the scores
-    __shared__ __align__(16) __nv_bfloat16 qsb[MT][D];  // bf16(phi(q))
-    __shared__ float A[MT][MT];                      // A[t][s] = q_t . k_s, s <= t
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ uint32_t tmem_holder;
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, int* status) {
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kWaitTimeoutNs) {
+            atomicExch(status, kStatusTimeout);
+            return false;
+        }
+    }
+    return true;
+}
 
-    const long u = blockIdx.x;
+__global__ void __launch_bounds__(vtf::THREADS, 1)
+verify_tf32_kernel(const __grid_constant__ CUtensorMap ms, const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                   __nv_bfloat16* __restrict__ o, long U, int m, int phi, int* status) {
+    using namespace vtf;
+    extern __shared__ uint8_t raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [SLOTS]
+    uint64_t* mma_bar = full + SLOTS;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(full + SLOTS + 1);
+    float* kf = reinterpret_cast<float*>(sm + OFF_KF);
+    float* A = reinterpret_cast<float*>(sm + OFF_A);
+    const uint32_t qt = smem_u32(sm + OFF_QT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const float4* Su = reinterpret_cast<const float4*>(S + u * D * D);
-    // S_0 -> bf16 tile: warp w converts rows w, w + 4, ...; lane c holds columns 4c .. 4c + 3
-    {
-        const int c = lane;
-        const uint32_t panel = static_cast<uint32_t>(c >> 4) * PANEL_S;
-        const uint32_t chunk = static_cast<uint32_t>((c & 15) >> 1), half = static_cast<uint32_t>(c & 1) * 8u;
-        const uint32_t sb = smem_u32(s_tile) + panel + half;
-#pragma unroll 4
-        for (int r0 = 0; r0 < D; r0 += 32) {
-            float4 x[8];
+    const uint32_t row_bytes = static_cast<uint32_t>(m) * D * 2;
+
+    // thread 32: S_0 and v of unit n of this CTA into slot n % SLOTS
+    auto issue = [&](long n) {
+        const long u = blockIdx.x + n * gridDim.x;
+        if (u >= U) return;
+        const int sl = static_cast<int>(n % SLOTS);
+        uint8_t* dst = sm + sl * SLOT;
+        mbar_arrive_expect_tx(&full[sl], SLOT_S + row_bytes);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = __ldcs(Su + (long)(r0 + 4 * j + warp) * (D / 4) + c);
+        for (int p = 0; p < 4; ++p) tma_load_3d(dst + p * PANEL_S, &ms, &full[sl], 32 * p, 0, static_cast<int>(u));
+        bulk_load(dst + SLOT_S, v + u * static_cast<long>(m) * D, row_bytes, &full[sl]);
+    };
+    // every thread: its 8-value pieces of the q and k rows of unit u
+    uint4 pq[2], pk[2];
+    auto fetch = [&](long u) {
+        if (u >= U) return;
+        const uint4* q4 = reinterpret_cast<const uint4*>(q + u * static_cast<long>(m) * D);
+        const uint4* k4 = reinterpret_cast<const uint4*>(k + u * static_cast<long>(m) * D);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t row = static_cast<uint32_t>(r0 + 4 * j + warp);
-                const uint32_t a = sb + row * 128u + ((chunk ^ (row & 7u)) << 4);
-                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a), "r"(pack_bf16x2(x[j].x, x[j].y)),
-                             "r"(pack_bf16x2(x[j].z, x[j].w))
-                             : "memory");
+        for (int r = 0; r < 2; ++r) {
+            const int e = tid * 8 + r * THREADS * 8;
+            if (e < m * D) {
+                pq[r] = __ldcs(q4 + e / 8);
+                pk[r] = __ldcs(k4 + e / 8);
             }
         }
-    }
-    // the drafts: phi(q) as a K-major bf16 tile and in fp32, phi(k) and v in fp32
-    const long base = u * (long)m * D;
-    for (int e = tid * 8; e < MT * D; e += TC_THREADS * 8) {
-        const int t = e / D, i = e % D;
-        float qv[8], kv[8];
-        if (t < m) {
-            unpack16(*reinterpret_cast<const uint4*>(q + base + e), qv);
-            unpack16(*reinterpret_cast<const uint4*>(k + base + e), kv);
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                qv[jj] = apply_phi(qv[jj], phi);
-                kv[jj] = apply_phi(kv[jj], phi);
-            }
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) qv[jj] = kv[jj] = 0.f;
-        }
-        const uint4 qp = make_uint4(pack_bf16x2(qv[0], qv[1]), pack_bf16x2(qv[2], qv[3]), pack_bf16x2(qv[4], qv[5]),
-                                    pack_bf16x2(qv[6], qv[7]));
-        *reinterpret_cast<uint4*>(&qsb[t][i]) = qp;
-        *reinterpret_cast<uint4*>(&ksb[t][i]) = make_uint4(pack_bf16x2(kv[0], kv[1]), pack_bf16x2(kv[2], kv[3]),
-                                                           pack_bf16x2(kv[4], kv[5]), pack_bf16x2(kv[6], kv[7]));
-        // the same 8 bf16 of row t, key dims i .. i + 7, as one 16-byte chunk of the K-major tile
-        const uint32_t qa = smem_u32(q_tile) + static_cast<uint32_t>(i >> 6) * PANEL_Q + static_cast<uint32_t>(t) * 128u +
-                            ((static_cast<uint32_t>((i & 63) >> 3) ^ static_cast<uint32_t>(t & 7)) << 4);
-        st_shared_v4(qa, qp.x, qp.y, qp.z, qp.w);
-    }
-    fence_proxy_async_smem();
+    };
+
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        prefetch_tmap(&ms);
+        for (int i = 0; i < SLOTS; ++i) mbar_init(&full[i], 1);
+        mbar_init(mma_bar, 1);
         fence_barrier_init();
     }
+    // draft rows m .. 15 of the B tile stay zero
+    for (uint32_t e = tid * 16; e < 4 * PANEL_Q; e += THREADS * 16) st_shared_v4(qt + e, 0, 0, 0, 0);
     if (warp == 0) {
-        tmem_alloc(&tmem_holder, 32);
+        tmem_alloc(tmem_holder, 32);
         tmem_relinquish();
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = tmem_holder;
-    if (tid == 0) {
-        constexpr uint32_t id = idesc_bf16(128, MT, 1, 0);  // A = bf16(S_0)^T MN-major, B = Q^T K-major
-        const uint64_t da = sw128_desc(smem_u32(s_tile), PANEL_S, 1024);
-        const uint64_t db = sw128_desc(smem_u32(q_tile), 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a_step = static_cast<uint64_t>(kk) * (2048u >> 4);
-            const uint64_t b_step = static_cast<uint64_t>((static_cast<uint32_t>(kk >> 2) * PANEL_Q + static_cast<uint32_t>(kk & 3) * 32u) >> 4);
-            mma_ss(tbase, da + a_step, db + b_step, id, kk > 0);
-        }
-        mma_commit(&bar);
-    }
-    // intra-draft scores while the product runs: one warp per pair (t, s), s <= t
-    {
-        int t = 0, s = warp;
-        while (s > t) { s -= t + 1; ++t; }
-        for (; t < m;) {
-            float a = 0.f;
-#pragma unroll
-            for (int i = lane; i < D; i += 32) a = fmaf(__bfloat162float(qsb[t][i]), __bfloat162float(ksb[s][i]), a);
-#pragma unroll
-            for (int off = 16; off; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-            if (lane == 0) A[t][s] = a;
-            s += TC_THREADS / 32;
-            while (s > t) { s -= t + 1; ++t; }
-        }
-    }
-    __syncthreads();
-    // O^T column j = tid: 16 drafts from TMEM (lane j), then the intra-draft terms
+    const uint32_t tbase = *tmem_holder;
+    if (tid == 32)
+        for (int i = 0; i < SLOTS; ++i) issue(i);
+    fetch(blockIdx.x);
+    constexpr uint32_t idesc = idesc_tf32(128, MT, 1, 0);  // A = S_0^T MN-major, B = Q^T K-major
+    long n = 0;
     bool ok = true;
-    {
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(&bar, 0)) {
-            if (globaltimer() - t0 > kWaitTimeoutNs) {
-                atomicExch(status, kStatusTimeout);
-                ok = false;
-                break;
+    for (;; ++n) {
+        const long u = blockIdx.x + n * gridDim.x;
+        if (u >= U) break;
+        const int sl = static_cast<int>(n % SLOTS);
+        // phi(q) into the swizzled B tile, phi(k) into kf (8 values a piece)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = tid * 8 + r * THREADS * 8;
+            if (e < m * D) {
+                const int t = e >> 7, i = e & (D - 1);
+                float x[8], y[8];
+                unpack16(pq[r], x);
+                unpack16(pk[r], y);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    x[jj] = apply_phi(x[jj], phi);
+                    y[jj] = apply_phi(y[jj], phi);
+                }
+                float4* kr = reinterpret_cast<float4*>(kf + e);
+                kr[0] = make_float4(y[0], y[1], y[2], y[3]);
+                kr[1] = make_float4(y[4], y[5], y[6], y[7]);
+                const uint32_t qa = qt + static_cast<uint32_t>(i >> 5) * PANEL_Q + static_cast<uint32_t>(t) * 128u;
+                const uint32_t c0 = static_cast<uint32_t>((i & 31) >> 2), sw = static_cast<uint32_t>(t & 7);
+                st_shared_v4(qa + ((c0 ^ sw) << 4), __float_as_uint(x[0]), __float_as_uint(x[1]),
+                             __float_as_uint(x[2]), __float_as_uint(x[3]));
+                st_shared_v4(qa + (((c0 + 1) ^ sw) << 4), __float_as_uint(x[4]), __float_as_uint(x[5]),
+                             __float_as_uint(x[6]), __float_as_uint(x[7]));
             }
         }
+        fetch(u + gridDim.x);
+        ok = wait_bounded(&full[sl], static_cast<uint32_t>((n / SLOTS) & 1), status);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (!__syncthreads_and(ok)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        if (tid == 0) {
+            // S_0 panels: 32 value columns x 128 key rows, 4-row groups 512 bytes apart
+            const uint64_t da = sw128b32_desc(smem_u32(sm + sl * SLOT), PANEL_S, 512);
+            const uint64_t db = sw128_desc(qt, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < D / 8; ++kk) {
+                // K = 8 per product: 8 key rows (1 KB) of the S_0 panels, 32 bytes of a Q row
+                const uint64_t a_step = static_cast<uint64_t>(kk) * (1024u >> 4);
+                const uint64_t b_step =
+                    static_cast<uint64_t>((static_cast<uint32_t>(kk >> 2) * PANEL_Q + static_cast<uint32_t>(kk & 3) * 32u) >> 4);
+                mma_ss_tf32(tbase, da + a_step, db + b_step, idesc, kk > 0);
+            }
+            mma_commit(mma_bar);
+        }
+        // intra-draft scores while the product runs, on threads 32 .. 111 (not
+        // the one issuing it): the lower triangle of 4 x 4 blocks of (t, s),
+        // 8 threads a block, each over the key dims 4 (p + 8 c) .. + 3,
+        // c = 0 .. 3 (so the 8 threads of a shared-memory phase read 8
+        // different bank groups), summed across the 8 by shuffles
+        {
+            const int w = tid - 32;
+            if (w >= 0 && w < 80) {
+                int tb = 0, sb = w >> 3;
+                while (sb > tb) {
+                    sb -= tb + 1;
+                    ++tb;
+                }
+                const int part = w & 7;
+                if (4 * tb < m) {
+                    float acc[4][4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t cc = static_cast<uint32_t>(part + 8 * c);
+                        float4 xa[4], yb[4];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const uint32_t t = static_cast<uint32_t>(4 * tb + a);
+                            const uint4 x = ld_shared_v4(qt + (cc >> 3) * PANEL_Q + t * 128u + (((cc & 7u) ^ (t & 7u)) << 4));
+                            xa[a] = make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z),
+                                                __uint_as_float(x.w));
+                        }
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) yb[b] = reinterpret_cast<const float4*>(kf + (4 * sb + b) * D)[cc];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                acc[a][b] = fmaf(xa[a].x, yb[b].x, acc[a][b]);
+                                acc[a][b] = fmaf(xa[a].y, yb[b].y, acc[a][b]);
+                                acc[a][b] = fmaf(xa[a].z, yb[b].z, acc[a][b]);
+                                acc[a][b] = fmaf(xa[a].w, yb[b].w, acc[a][b]);
+                            }
+                    }
+                    const unsigned grp = 0xFFu << (lane & 24);
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            float x = acc[a][b];
+                            x += __shfl_xor_sync(grp, x, 4);
+                            x += __shfl_xor_sync(grp, x, 2);
+                            x += __shfl_xor_sync(grp, x, 1);
+                            acc[a][b] = x;
+                        }
+                    if (part == 0)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            *reinterpret_cast<float4*>(A + (4 * tb + a) * MT + 4 * sb) =
+                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+                }
+            }
+        }
+        __syncthreads();
+        ok = wait_bounded(mma_bar, static_cast<uint32_t>(n & 1), status);
+        if (!__syncthreads_and(ok)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld16(tbase + (static_cast<uint32_t>(warp * 32) << 16), r);
+        {
+            const int j = tid;
+            const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(sm + sl * SLOT + SLOT_S);
+            float vj[MT];
+#pragma unroll
+            for (int s = 0; s < MT; ++s) vj[s] = s < m ? __bfloat162float(vs[s * D + j]) : 0.f;
+            tmem_wait_ld();
+            const long base = u * static_cast<long>(m) * D;
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                if (t < m) {
+                    float y = __uint_as_float(r[t]);
+                    const float4* a4 = reinterpret_cast<const float4*>(A + t * MT);
+#pragma unroll
+                    for (int s4 = 0; s4 <= t / 4; ++s4) {
+                        const float4 a = a4[s4];
+                        y = fmaf(a.x, vj[4 * s4], y);
+                        if (4 * s4 + 1 <= t) y = fmaf(a.y, vj[4 * s4 + 1], y);
+                        if (4 * s4 + 2 <= t) y = fmaf(a.z, vj[4 * s4 + 2], y);
+                        if (4 * s4 + 3 <= t) y = fmaf(a.w, vj[4 * s4 + 3], y);
+                    }
+                    o[base + static_cast<long>(t) * D + j] = __float2bfloat16_rn(y);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 32) issue(n + SLOTS);
     }
-    tc_fence_after();
-    uint32_t r[16];
-    tmem_ld16(tbase + (static_cast<uint32_t>(warp * 32) << 16), r);
-    tmem_wait_ld();
-    if (ok) {
-        const int j = tid;
-        float vj[MT];
-#pragma unroll
-        for (int s = 0; s < MT; ++s) vj[s] = s < m ? __bfloat162float(v[base + (long)s * D + j]) : 0.f;
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            if (t < m) {
-                float y = __uint_as_float(r[t]);
-#pragma unroll
-                for (int s = 0; s <= t; ++s) y = fmaf(A[t][s], vj[s], y);
-                o[base + (long)t * D + j] = __float2bfloat16_rn(y);
-            }
-        }
+    if (!ok && tid == 32) {
+        // copies still in flight land before the CTA's shared memory is released
+        for (long x = n; x < n + SLOTS; ++x)
+            if (blockIdx.x + x * gridDim.x < U)
+                if (!wait_bounded(&full[x % SLOTS], static_cast<uint32_t>((x / SLOTS) & 1), status)) break;
     }
     tc_fence_before();
     __syncthreads();

@@ -153,6 +153,9 @@ la_status device_info(DeviceInfo** out) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tcw::SMEM_BYTES)) !=
                 cudaSuccess)
                 return cuda_fail(e, "cudaFuncSetAttribute(prefill_wide)");
+        if ((e = cudaFuncSetAttribute(dmulti::verify_tf32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      dmulti::vtf::SMEM_BYTES)) != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(verify_tf32)");
         if ((e = set_simt_attrs<float>()) != cudaSuccess || (e = set_simt_attrs<__nv_bfloat16>()) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
         const unsigned long long id = current_ctx_id();
@@ -191,6 +194,24 @@ la_status make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, u
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LA_OK;
+}
+
+// U fp32 d x d states, row-major and back to back, as a 3-D map {d, d, U} with
+// boxes of 32 columns x d rows x 1 unit (128 bytes a row, 128-byte swizzle of
+// 32-byte atoms: the MN-major tf32 operand layout).
+la_status make_state_map(CUtensorMap* m, const float* S, uint64_t d, uint64_t U) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    la_status s = encoder(&enc);
+    if (s != LA_OK) return s;
+    cuuint64_t dims[3] = {d, d, U};
+    cuuint64_t strides[2] = {d * 4, d * d * 4};
+    cuuint32_t box[3] = {32, static_cast<cuuint32_t>(d), 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(S), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled (state) failed (%d)", (int)r);
     return LA_OK;
 }
 
@@ -920,12 +941,12 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o, f
 }
 
 // Drafts up to which the FFMA verify kernel is the faster one (measured at
-// B=256, H=64, d=128, bf16, ms, FFMA / tensor cores: m = 1 0.154 / 0.277,
-// m = 4 0.164 / 0.284, m = 8 0.242 / 0.328, m = 12 0.391 / 0.396, m = 16
-// 0.584 / 0.456): the tensor-core kernel has a higher fixed cost per unit
-// (its S_0 load and conversion do not overlap its product), but its cost
-// grows less with m.
-constexpr int kVerifyFfmaMaxM = 12;
+// B=256, H=64, d=128, bf16, ms, FFMA / tensor cores: m = 1 0.153 / 0.206,
+// m = 4 0.164 / 0.215, m = 8 0.242 / 0.225, m = 12 0.392 / 0.241, m = 16
+// 0.584 / 0.261): below that the FFMA kernel streams the state at the HBM
+// rate and the tensor-core kernel's per-unit chain (16 tf32 products, TMEM
+// read-back) is longer than a unit's share of the bandwidth.
+constexpr int kVerifyFfmaMaxM = 4;
 
 la_status la_decode_verify(const void* q, const void* k, const void* v, void* o, const float* S, int B, int H,
                            int m, int dk, int dv, la_dtype dt, la_phi phi, la_stream_t stream) {
@@ -944,17 +965,24 @@ la_status la_decode_verify(const void* q, const void* k, const void* v, void* o,
     DeviceInfo* di;
     if ((s = device_info(&di)) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // bf16 at d = 128: the q S_0 products on the tensor cores once the drafts
-    // make the FFMA kernel compute-bound (LA_VERIFY_TC=1 / 0 forces it on / off)
+    // bf16 at d = 128: the q S_0 products on the tensor cores (tf32 reads of
+    // the fp32 state) beyond kVerifyFfmaMaxM drafts (LA_VERIFY_TC=1 / 0
+    // forces them on / off)
     bool tcv = dt == LA_BF16 && dk == 128 && m > kVerifyFfmaMaxM;
     if (dt == LA_BF16 && dk == 128)
         if (const char* e = getenv("LA_VERIFY_TC")) tcv = e[0] == '1';
-    if (tcv)
-        dmulti::verify_tc_kernel<<<(int)U, dmulti::TC_THREADS, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
-            reinterpret_cast<const __nv_bfloat16*>(v), reinterpret_cast<__nv_bfloat16*>(o), S, m, phi, di->status);
-    else if (dt == LA_BF16) launch_verify<__nv_bfloat16>(dk, m, (int)U, q, k, v, o, S, phi, st);
-    else launch_verify<float>(dk, m, (int)U, q, k, v, o, S, phi, st);
+    if (tcv) {
+        CUtensorMap ms;
+        if ((s = make_state_map(&ms, S, 128, (uint64_t)U)) != LA_OK) return s;
+        const int grid = (int)std::min<long>(U, di->sms);
+        dmulti::verify_tf32_kernel<<<grid, dmulti::vtf::THREADS, dmulti::vtf::SMEM_BYTES, st>>>(
+            ms, reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
+            reinterpret_cast<const __nv_bfloat16*>(v), reinterpret_cast<__nv_bfloat16*>(o), U, m, phi, di->status);
+    } else if (dt == LA_BF16) {
+        launch_verify<__nv_bfloat16>(dk, m, (int)U, q, k, v, o, S, phi, st);
+    } else {
+        launch_verify<float>(dk, m, (int)U, q, k, v, o, S, phi, st);
+    }
     return after_launch("decode_verify launch");
 }
 

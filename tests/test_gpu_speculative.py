@@ -24,7 +24,7 @@ def la():
 
 def _case(B, H, m, d, dtype, seed):
     U = B * H
-    S = synth.outer_product_state(U, d, d, [3000 + 100 * u for u in range(U)], seed=seed).view(B, H, d, d)
+    S = synth.outer_product_state(U, d, d, [3000 + 100 * (u % 12) for u in range(U)], seed=seed).view(B, H, d, d)
     q, k, v = synth.qkv((B, H, m, d), d, dtype, seed=seed + 1)
     return S, q, k, v
 
@@ -45,12 +45,13 @@ def test_verify_matches_recurrence_over_drafts(la, oracle_mod, m, d, dtype):
 
 @pytest.mark.parametrize("m", [1, 3, 4, 5, 8, 13, 16])
 @pytest.mark.parametrize("phi", ["identity", "relu", "elu1"])
-def test_verify_tensor_cores_match_recurrence(la, oracle_mod, monkeypatch, m, phi):
-    """bf16 at d = 128 with the q S_0 products on the tensor cores (bf16(S_0)
-    as the operand, fp32 accumulation), forced for every m: the fp64
-    recurrence over the drafts at the bf16 output bars, and the FFMA kernel
-    (fp32 S_0) within the same bars."""
-    B, H, d = 3, 4, 128
+@pytest.mark.parametrize("B,H", [(3, 4), (2, 200)])  # 12 units; 400 units, several per CTA of the persistent grid
+def test_verify_tensor_cores_match_recurrence(la, oracle_mod, monkeypatch, m, phi, B, H):
+    """bf16 at d = 128 with the q S_0 products on the tensor cores (the fp32
+    S_0 read as tf32, fp32 accumulation), forced for every m: the fp64
+    recurrence over the drafts at the bf16 output bars, per unit, and the
+    FFMA kernel (fp32 S_0) within the same bars."""
+    d = 128
     S, q, k, v = _case(B, H, m, d, "bf16", seed=m * 7 + 1)
     Sd = S.cuda()
     monkeypatch.setenv("LA_VERIFY_TC", "1")
