@@ -536,13 +536,31 @@ def run_config1(args, dist: Dist, pk, cpu=False):
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     n = 200
-    total_ms, _ = timed_launches(lambda: la.prefill(q, k, v, None, out=o, s_out=s, chunk=64), n,
-                                 max(3, args.warmup), dist, stream)
+    call = lambda: la.prefill(q, k, v, None, out=o, s_out=s, chunk=64)
+    total_ms, _ = timed_launches(call, n, max(3, args.warmup), dist, stream)
     ms_step = dist.max(total_ms) / n
+    # the same call captured in a CUDA graph (64 calls a replay): the device's
+    # own time per call, without the Python binding's per-call host work
+    calls = 64
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call()
+    stream.wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            call()
+    reps = 10
+    g_ms, _ = timed_launches(g.replay, reps, max(3, args.warmup), dist, stream)
+    g_step = dist.max(g_ms) / (reps * calls)
+    del g
     res = dict(workload="prefill B=1 H=2 N=256 d=64 fp32, chunk 64, zero initial state (FFMA path)",
                us_per_step=ms_step * 1e3, tokens_per_s=B * N * dist.world / (ms_step / 1e3),
                tflops_rec=flops_rec(B * H * N, d) / (ms_step / 1e3) / 1e12, steps=n,
-               l2="inputs (256 KiB) stay in L2: a latency figure")
+               graph_us_per_call=g_step * 1e3, tokens_per_s_graph=B * N * dist.world / (g_step / 1e3),
+               l2="inputs (256 KiB) stay in L2: a latency figure; us_per_step is one Python call back to back, "
+                  "graph_us_per_call the device time of a call replayed from a CUDA graph")
     if cpu:
         res["cpu_baseline"] = oracle_dense_baseline(q.cpu(), k.cpu(), v.cpu(), 1, "the whole workload", reps=50)
     del q, k, v, o, s
@@ -818,7 +836,7 @@ def summary_line(extras):
     pick("decode", "decode_fp32_state", ("hbm_gbs", "frac", "ms_per_step", "tokens_per_s"))
     pick("varlen", "varlen_resume", ("tokens_per_s", "ms_per_step", "hbm_gbs", "frac"))
     pick("prefill_8k", "prefill_8k", ("tokens_per_s", "ms_per_step", "hbm_gbs", "frac"))
-    pick("config1_fp32", "config1_fp32", ("us_per_step", "tokens_per_s", "tflops_rec"))
+    pick("config1_fp32", "config1_fp32", ("us_per_step", "graph_us_per_call", "tokens_per_s", "tflops_rec"))
     pick("backward_8k", "backward_8k", ("ms_per_step", "hbm_gbs", "frac"))
     pick("speculative_m16", "verify_m16", ("ms_verify", "verify_hbm_gbs", "verify_frac"))
     return out

@@ -415,9 +415,19 @@ namespace {
 // remains.  LA_PREFILL_SEGMENTS=<n> overrides the count (1 = no split).
 constexpr int kMinSegChunks = 8;
 
-int plan_segments(long U, int N, int slices, int sms, int* seg_len) {
-    const int nch = (N + tc::C - 1) / tc::C;
-    *seg_len = nch * tc::C;
+// On the FFMA path a chunk is compute-heavy (about 4 C d^2 FMAs on one SM), so
+// there a segment of a single chunk already pays for its share of the
+// state-only pass once the units leave SMs idle (fp32, B=1, H=2, N=256, d=64,
+// chunk 64: 44 us a call unsplit, on 2 SMs).
+constexpr int kMinSegChunksSimt = 1;
+constexpr int kSimtSmallestChunk = 32;
+
+// Segments are whole chunks of `unit` tokens (the tensor-core tile, or the
+// FFMA kernel's chunk), at least min_chunks of them.
+int plan_segments(long U, int N, int slices, int sms, int* seg_len, int unit = tc::C,
+                  int min_chunks = kMinSegChunks) {
+    const int nch = (N + unit - 1) / unit;
+    *seg_len = nch * unit;
     if (N <= 0) return 1;
     int P;
     if (const char* e = getenv("LA_PREFILL_SEGMENTS")) {
@@ -425,12 +435,19 @@ int plan_segments(long U, int N, int slices, int sms, int* seg_len) {
     } else {
         const long items = U * slices;
         P = items * 2 > sms ? 1 : (int)(sms / items);
-        P = std::min(P, nch / kMinSegChunks);
+        P = std::min(P, nch / min_chunks);
     }
     P = std::max(1, std::min(P, nch));
     const int cps = (nch + P - 1) / P;  // chunks per segment
-    *seg_len = cps * tc::C;
+    *seg_len = cps * unit;
     return (nch + cps - 1) / cps;
+}
+
+// The most segments an FFMA-path call may plan (its chunk is not known to the
+// workspace queries; the smallest chunk gives the most segments).
+int plan_segments_simt_max(long U, int N, int sms) {
+    int seg_len;
+    return plan_segments(U, N, 1, sms, &seg_len, kSimtSmallestChunk, kMinSegChunksSimt);
 }
 
 size_t segment_workspace_bytes(long U, int P, int dk, int dv) {
@@ -492,7 +509,7 @@ la_status simt_dense(const void* q, const void* k, const void* v, void* o, const
                              : launch_simt<__nv_bfloat16>(d, chunk, (int)grid, q, k, v, o, x, st);
     };
     int seg_len;
-    int P = plan_segments(U, N, 1, di->sms, &seg_len);
+    int P = plan_segments(U, N, 1, di->sms, &seg_len, chunk ? chunk : kSimtDefaultChunk, kMinSegChunksSimt);
     if (P > 1 && (!ws || ws_bytes < segment_workspace_bytes(U, P, d, d) || !aligned16(ws) || U * P > (1L << 30)))
         P = 1;
     if (P <= 1) return go(sp, U);
@@ -532,8 +549,10 @@ size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtyp
     DeviceInfo* di;
     if (device_info(&di) != LA_OK) return ph;
     int seg_len;
-    const int P = plan_segments(U, N, tc ? tc_slices(dk) : 1, di->sms, &seg_len);
-    const size_t seg = segment_workspace_bytes(U, P, dk, dv);
+    // (a bf16 call with 32- or 64-token chunks runs on the FFMA path; sized for
+    // the tensor-core plan, its workspace may leave it unsplit)
+    const size_t seg = tc ? segment_workspace_bytes(U, plan_segments(U, N, tc_slices(dk), di->sms, &seg_len), dk, dv)
+                          : segment_workspace_bytes(U, plan_segments_simt_max(U, N, di->sms), dk, dv);
     return ph ? round256(seg) + ph : seg;
 }
 
@@ -1141,8 +1160,8 @@ size_t la_prefill_backward_workspace_size(int B, int H, int N, int d_k, int d_v,
     if (device_info(&di) != LA_OK) return 0;
     int seg_len;
     const long U = (long)B * H;
-    const int slices = use_tensor_cores(d_k, dt) ? tc_slices(d_k) : 1;
-    return segment_workspace_bytes(U, plan_segments(U, N, slices, di->sms, &seg_len), d_k, d_v);
+    if (!use_tensor_cores(d_k, dt)) return segment_workspace_bytes(U, plan_segments_simt_max(U, N, di->sms), d_k, d_v);
+    return segment_workspace_bytes(U, plan_segments(U, N, tc_slices(d_k), di->sms, &seg_len), d_k, d_v);
 }
 
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout, const float* s0,

@@ -178,11 +178,48 @@ def test_ffma_segments_with_phi(la, oracle_mod, monkeypatch, phi):
     assert_state(s.cpu(), rs, 2)
 
 
+@pytest.mark.parametrize("N,chunk", [(256, 64), (256, 32), (100, 32), (64 + 5, 64), (64, 64), (1, 32)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_ffma_short_sequences_split_by_chunk(la, oracle_mod, N, chunk, d):
+    """Short sequences on few units are cut into segments of whole FFMA chunks
+    (one chunk each at the least), from the given start state; ragged tails
+    included."""
+    B, H = 1, 2
+    q, k, v = synth.dense(B, H, N, d, "fp32", seed=N + chunk + d)
+    s0 = _state(B, H, d, seed=N + 3)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), s0.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    assert_out(o.cpu(), ro, torch.float32, 2)
+    assert_state(s.cpu(), rs, 2)
+
+
+@pytest.mark.parametrize("chunk", [32, 64])
+@pytest.mark.parametrize("segments", [None, "1"])
+def test_ffma_short_sequences_integer_inputs_bit_exact(la, oracle_mod, monkeypatch, chunk, segments):
+    """The chunk-sized segments of a short sequence, and the unsplit run, give
+    the oracle's result bit for bit on integer-valued inputs."""
+    if segments:
+        monkeypatch.setenv("LA_PREFILL_SEGMENTS", segments)
+    B, H, N, d = 1, 2, 256 + 17, 64
+    q, k, v = (synth.integer_valued((B, H, N, d), seed=s) for s in (71, 72, 73))
+    s0 = synth.integer_valued((B, H, d, d), seed=74, lo=-20, hi=20)
+    o, s = la.prefill(q.cuda(), k.cuda(), v.cuda(), s0.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.device_status() == 0
+    ro, rs = oracle_mod.recurrent(q, k, v, s0)
+    np.testing.assert_array_equal(to64(o.cpu()), ro)
+    np.testing.assert_array_equal(to64(s.cpu()), rs)
+
+
 def test_ffma_workspace_size_follows_the_plan(la):
     # one item per unit on the FFMA path: 128 units fill the GPU, 8 do not
     assert la.prefill_workspace_size(1, 128, 65536, 128, torch.float32) == 0
     n = la.prefill_workspace_size(1, 8, 65536, 128, torch.float32)
     assert n > 0 and n % (8 * 128 * 128 * 4) == 0
+    # a short sequence on few units is split too (segments of whole FFMA chunks)
+    assert la.prefill_workspace_size(1, 2, 256, 64, torch.float32) > 0
 
 
 def _varlen_case(lens, H, d, seed, dtype="fp32", n_pool=2):
