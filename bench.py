@@ -53,8 +53,8 @@ METRIC = "prefill tokens/s & % bf16 tensor peak at N=128K; decode-step HBM GB/s"
 # with the token-head count, so a launch is scaled by its token-heads.  When the
 # kernel sources change the figure no longer applies and is reported as null.
 TRAFFIC_SOURCES = ("long_context_linear_b200/csrc/prefill_tc.cuh", "long_context_linear_b200/csrc/sm100.cuh")
-TRAFFIC_HASH = "1c63d16b44b4bc9e"
-TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.72256e6 + 114.2464e6) / (16 * 32768)
+TRAFFIC_HASH = "f327651e3f2dcfb9"
+TRAFFIC_BYTES_PER_TOKEN_HEAD = (402.712576e6 + 113.398784e6) / (16 * 32768)
 
 
 # ----------------------------------------------------------------- helpers
