@@ -497,8 +497,8 @@ def run_prefill8k(args, dist: Dist, pk, phi: str = "identity", d: int = 0, cpu=F
     q, k, v = synth.dense(B, H, N, d, "bf16", seed=61 + dist.rank, device=dev)
     o = torch.empty_like(v)
     s = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    # with elu + 1 the workspace holds phi(q), phi(k) (mapped by a pre-pass);
-    # relu is mapped on the tiles inside the prefill kernel
+    # the library sizes the workspace: at this shape (full-width kernel) relu
+    # and elu + 1 are both mapped on the tiles inside the prefill kernel
     ws_bytes = la.prefill_workspace_size(B, H, N, d, torch.bfloat16, phi)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)

@@ -119,12 +119,15 @@ LA_API int la_version(void);
  * N = 0 writes s_out = s0 (or zero).  Returns LA_OK once enqueued.
  */
 LA_API size_t la_prefill_workspace_size(int B, int H, int N, int dk, int dv, la_dtype dt);
-/* The same for la_prefill_ex with feature map `phi`: on the tensor-core path
- * elu + 1 adds room for phi(q) and phi(k) (2 x B*H*N*dk bf16, each rounded up
- * to 256 bytes) after the segment states; given that room the call maps q and
- * k in one bandwidth-bound pass first, otherwise the prefill kernel maps the
- * tiles in shared memory (same results, slower).  relu is always mapped in the
- * kernel (faster than a separate pass) and adds nothing. */
+/* The same for la_prefill_ex with feature map `phi`.  When the (batch, head)
+ * units fill fewer than half of the SMs (two CTAs per head on the tensor-core
+ * path), elu + 1 adds room for phi(q) and phi(k) (2 x B*H*N*dk bf16, each
+ * rounded up to 256 bytes) after the segment states; given that room the call
+ * maps q and k in one bandwidth-bound pass first, otherwise the prefill kernel
+ * maps the tiles in shared memory (same results, slower there).  With more
+ * units (one CTA per head) the kernel maps elu + 1 itself, a chunk ahead, and
+ * nothing is added (environment variable LA_PHI_PREPASS=1 keeps the pass and
+ * its room there too).  relu is always mapped in the kernel and adds nothing. */
 LA_API size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtype dt, la_phi phi);
 LA_API la_status la_prefill(const void* q, const void* k, const void* v, void* o,
                      const float* s0, float* s_out,
@@ -154,8 +157,8 @@ LA_API la_status la_prefill_ex(const void* q, const void* k, const void* v, void
  */
 LA_API size_t la_prefill_varlen_workspace_size(int n_seq, int T, int H, int dk, int dv, la_dtype dt);
 /* The same for la_prefill_varlen_ex with feature map `phi`: with elu + 1 adds
- * room for phi(q) and phi(k) (2 x T*H*dk bf16) after the order array, used as
- * for the dense call. */
+ * room for phi(q) and phi(k) (2 x T*H*dk bf16) after the order array, on the
+ * same terms as the dense call (n_seq x H units). */
 LA_API size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int dv, la_dtype dt,
                                                   la_phi phi);
 LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v, void* o,

@@ -466,6 +466,13 @@ size_t phi_workspace_bytes(long rows, int d, la_phi phi) {
     return 2 * round256((size_t)rows * (size_t)d * 2);
 }
 
+// elu + 1 through the pre-pass only on the value-split kernel, whose two
+// CTAs of a head would both map the tiles; the full-width kernel maps them
+// once per head, a chunk ahead (B=4, H=32, N=8K: 0.31-0.33 ms mapped in the
+// kernel against 0.36 ms with the pre-pass).  LA_PHI_PREPASS=1 keeps the
+// pre-pass on the full-width kernel too (the two routes are tested equal).
+bool phi_prepass_wanted(bool wide) { return !wide || env_flag("LA_PHI_PREPASS"); }
+
 // phi over q and k (each `elems` bf16) into the two halves of `scratch`; on
 // success q and k are redirected to the mapped copies.
 la_status phi_prepass(const void** q, const void** k, void* scratch, long elems, la_phi phi, DeviceInfo* di,
@@ -545,9 +552,9 @@ size_t la_prefill_workspace_size_ex(int B, int H, int N, int dk, int dv, la_dtyp
     if (B <= 0 || H <= 0 || N <= 0 || dk != dv || (dk != 64 && dk != 128)) return 0;
     const bool tc = use_tensor_cores(dk, dt);
     const long U = (long)B * H;
-    const size_t ph = tc ? phi_workspace_bytes(U * N, dk, phi) : 0;
     DeviceInfo* di;
-    if (device_info(&di) != LA_OK) return ph;
+    if (device_info(&di) != LA_OK) return tc ? phi_workspace_bytes(U * N, dk, phi) : 0;
+    const size_t ph = tc && phi_prepass_wanted(use_wide(U, dk, di)) ? phi_workspace_bytes(U * N, dk, phi) : 0;
     int seg_len;
     // (a bf16 call with 32- or 64-token chunks runs on the FFMA path; sized for
     // the tensor-core plan, its workspace may leave it unsplit)
@@ -613,7 +620,8 @@ la_status la_prefill_ex(const void* q, const void* k, const void* v, void* o, co
     }
     // phi(q), phi(k) mapped up front when the workspace has room behind the
     // segment states; otherwise the kernel maps the tiles in shared memory
-    const size_t off_phi = P > 1 ? round256(ws_need) : 0, ws_phi = phi_workspace_bytes(U * N, dk, phi);
+    const size_t off_phi = P > 1 ? round256(ws_need) : 0;
+    const size_t ws_phi = phi_prepass_wanted(wide) ? phi_workspace_bytes(U * N, dk, phi) : 0;
     if (ws_phi && workspace && aligned16(workspace) && ws_bytes >= off_phi + ws_phi) {
         if ((s = phi_prepass(&q, &k, reinterpret_cast<uint8_t*>(workspace) + off_phi, U * N * dk, phi, di, st)) !=
             LA_OK)
@@ -713,9 +721,11 @@ size_t la_prefill_varlen_workspace_size_ex(int n_seq, int T, int H, int dk, int 
     const size_t base = varlen_order_bytes(n_seq);
     if (!base || T <= 0 || H <= 0 || dk != dv || (dk != 64 && dk != 128)) return base;
     const bool tc = use_tensor_cores(dk, dt);
-    size_t total = base + (tc ? phi_workspace_bytes((long)T * H, dk, phi) : 0);
     DeviceInfo* di;
-    if (device_info(&di) != LA_OK) return total;
+    if (device_info(&di) != LA_OK) return base + (tc ? phi_workspace_bytes((long)T * H, dk, phi) : 0);
+    size_t total = base + (tc && phi_prepass_wanted(use_wide((long)n_seq * H, dk, di))
+                               ? phi_workspace_bytes((long)T * H, dk, phi)
+                               : 0);
     int min_seg;
     const long max_segs = plan_varlen_segments(n_seq, T, H, tc ? tc_slices(dk) : 1, di->sms, &min_seg);
     if (max_segs) total += varlen_segment_bytes(n_seq, max_segs, H, dk);
@@ -830,7 +840,8 @@ la_status la_prefill_varlen_ex(const void* q, const void* k, const void* v, void
     int* order = reinterpret_cast<int*>(workspace);
     vorder::order_kernel<<<1, vorder::NUM_THREADS, 0, st>>>(cu_seqlens, n_seq, order);
     if ((s = after_launch("varlen order launch")) != LA_OK) return s;
-    const size_t ws_phi = T > 0 ? phi_workspace_bytes((long)T * H, dk, phi) : 0;
+    const size_t ws_phi =
+        T > 0 && phi_prepass_wanted(use_wide((long)n_seq * H, dk, di)) ? phi_workspace_bytes((long)T * H, dk, phi) : 0;
     size_t off_seg = need;
     if (ws_phi && ws_bytes >= need + ws_phi) {
         if ((s = phi_prepass(&q, &k, reinterpret_cast<uint8_t*>(workspace) + need, (long)T * H * dk, phi, di, st)) !=

@@ -549,19 +549,28 @@ prefill_wide_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
 #pragma unroll
                 for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
+            // phi(K), then phi(Q), of the chunk with global index gg (slot gg %
+            // SLOTS), in place, before the tensor cores read them
+            auto map_chunk = [&](long gg) -> bool {
+                const int sg = static_cast<int>(gg % SLOTS);
+                const uint32_t par = static_cast<uint32_t>((gg / SLOTS) & 1);
+                if (!tc::warp_wait(&k_full[sg], par, abort, p.status)) return false;
+                phi_tile2(smem_u32(sm + OFF_K + sg * TILE), tid, phi);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&kphi_full[sg]);
+                if (!tc::warp_wait(&q_full[sg], par, abort, p.status)) return false;
+                phi_tile2(smem_u32(sm + OFF_Q + sg * TILE), tid, phi);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qk_mapped[sg]);
+                return true;
+            };
+            // elu + 1 (exponentials) maps an item's later chunks a chunk ahead
+            // (below), so that the mapping is not queued behind the state
+            // update on the way to the next chunk's Q K^T; relu's packed max is
+            // cheap enough to map each chunk at its start
+            const bool ahead = phi == PHI_ELU1;
             for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
-                const int s = g % SLOTS;
-                if (kGeneral && phi != PHI_IDENTITY) {
-                    // phi(K_c) then phi(Q_c), in place, before the tensor cores read them
-                    if (!tc::warp_wait(&k_full[s], (g / SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                    phi_tile2(smem_u32(sm + OFF_K + s * TILE), tid, phi);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&kphi_full[s]);
-                    if (!tc::warp_wait(&q_full[s], (g / SLOTS) & 1, abort, p.status)) { stop = true; break; }
-                    phi_tile2(smem_u32(sm + OFF_Q + s * TILE), tid, phi);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&qk_mapped[s]);
-                }
+                if (kGeneral && phi != PHI_IDENTITY && (c0 == 0 || !ahead) && !map_chunk(g)) { stop = true; break; }
                 // publish bf16(S_{c-1})^T once Q S of the previous chunk has read the old one
                 if (g > 0 && !tc::warp_wait(st_free, (g - 1) & 1, abort, p.status)) { stop = true; break; }
 #pragma unroll
@@ -571,6 +580,7 @@ prefill_wide_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_full);
+                if (kGeneral && ahead && c0 + C < it.len && !map_chunk(g + 1)) { stop = true; break; }
                 // absorb dS_c
                 if (!tc::warp_wait(ds_full, g & 1, abort, p.status)) { stop = true; break; }
                 tc_fence_after();

@@ -207,9 +207,11 @@ def test_wide_relu_in_kernel_equals_identity_on_mapped_inputs(la, wide):
     assert torch.equal(s1, s2)
 
 
-def test_wide_elu1_in_kernel_equals_prepass(la, wide):
+def test_wide_elu1_in_kernel_equals_prepass(la, wide, monkeypatch):
     """elu + 1 mapped by the kernel (no workspace) and by the pre-pass
-    (workspace given) round phi to bf16 the same way: bit-identical."""
+    (workspace given, the pre-pass forced on the full-width kernel) round phi
+    to bf16 the same way: bit-identical."""
+    monkeypatch.setenv("LA_PHI_PREPASS", "1")
     B, H, N, d = 1, 2, 3000, 128
     q, k, v = synth.dense(B, H, N, d, "bf16", seed=95, device="cuda")
     ws = torch.empty(la.prefill_workspace_size(B, H, N, d, torch.bfloat16, "elu1"), dtype=torch.uint8,
@@ -227,6 +229,18 @@ def test_wide_elu1_in_kernel_equals_prepass(la, wide):
     assert la.device_status() == 0
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1], outs[1][1])
+
+
+def test_wide_elu1_needs_no_prepass_workspace(la):
+    """Shapes that run on the full-width kernel map elu + 1 in the kernel and
+    ask for no room for mapped copies of q and k."""
+    args = (4, 32, 8192, 128, torch.bfloat16)
+    assert la.prefill_workspace_size(*args, "elu1") == la.prefill_workspace_size(*args)
+    assert la.prefill_varlen_workspace_size(64, 64 * 1000, 32, 128, torch.bfloat16, "elu1") == \
+        la.prefill_varlen_workspace_size(64, 64 * 1000, 32, 128, torch.bfloat16)
+    # two heads run on the value split, where the pre-pass pays
+    assert la.prefill_workspace_size(1, 2, 3000, 128, torch.bfloat16, "elu1") > \
+        la.prefill_workspace_size(1, 2, 3000, 128, torch.bfloat16)
 
 
 @pytest.mark.parametrize("phi", ["relu", "elu1"])
