@@ -147,8 +147,9 @@ la_status device_info(DeviceInfo** out) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES)) !=
                 cudaSuccess)
                 return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
-        const void* wide_kernels[2] = {reinterpret_cast<const void*>(tcw::prefill_wide_kernel<false>),
-                                       reinterpret_cast<const void*>(tcw::prefill_wide_kernel<true>)};
+        const void* wide_kernels[3] = {reinterpret_cast<const void*>(tcw::prefill_wide_kernel<false>),
+                                       reinterpret_cast<const void*>(tcw::prefill_wide_kernel<true>),
+                                       reinterpret_cast<const void*>(tcw::prefill_wide_kernel<true, true>)};
         for (const void* kern : wide_kernels)
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tcw::SMEM_BYTES)) !=
                 cudaSuccess)
@@ -308,8 +309,12 @@ bool use_wide(long units, int d, const DeviceInfo* di) {
 la_status launch_wide(int grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mo, const tc::Params& p, cudaStream_t st, const char* what) {
     const bool general = p.phi != LA_PHI_IDENTITY || p.reverse || p.init_transposed;
-    if (general) tcw::prefill_wide_kernel<true><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
-    else tcw::prefill_wide_kernel<false><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    if (p.phi == LA_PHI_ELU1)
+        tcw::prefill_wide_kernel<true, true><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    else if (general)
+        tcw::prefill_wide_kernel<true><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    else
+        tcw::prefill_wide_kernel<false><<<grid, tcw::NUM_THREADS, tcw::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
     return after_launch(what);
 }
 

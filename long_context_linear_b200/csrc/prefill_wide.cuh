@@ -126,7 +126,10 @@ __device__ __forceinline__ void phi_tile2(uint32_t base, int t, int phi) {
 // given (the common forward case).  kGeneral = true adds the feature map on
 // the Q and K tiles, the reverse chunk order and the transposed initial state
 // of the backward passes.  Items are whole sequences (no segments).
-template <bool kGeneral>
+// kAhead (with kGeneral, for elu + 1): the state warps map each chunk's
+// tiles a chunk ahead (below); a separate instance, so that the others keep a
+// single mapping site in their loop.
+template <bool kGeneral, bool kAhead = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 prefill_wide_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -564,11 +567,11 @@ prefill_wide_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                 if (lane == 0) mbar_arrive(&qk_mapped[sg]);
                 return true;
             };
-            // elu + 1 (exponentials) maps an item's later chunks a chunk ahead
-            // (below), so that the mapping is not queued behind the state
-            // update on the way to the next chunk's Q K^T; relu's packed max is
-            // cheap enough to map each chunk at its start
-            const bool ahead = phi == PHI_ELU1;
+            // with kAhead (elu + 1: exponentials) an item's later chunks are
+            // mapped a chunk ahead (below), so that the mapping is not queued
+            // behind the state update on the way to the next chunk's Q K^T;
+            // relu's packed max is cheap enough to map each chunk at its start
+            constexpr bool ahead = kAhead;
             for (int c0 = 0; c0 < it.len; c0 += C, ++g) {
                 if (kGeneral && phi != PHI_IDENTITY && (c0 == 0 || !ahead) && !map_chunk(g)) { stop = true; break; }
                 // publish bf16(S_{c-1})^T once Q S of the previous chunk has read the old one
